@@ -1,0 +1,304 @@
+"""Pins for the CPU oracle: each test ties the oracle to something other than
+itself -- the binary16 format via numpy's converters, hand-worked values,
+invariants the method guarantees, the truncation bound against an exact
+GEMM computed by numpy, integer brute force -- so that a dropped term, a
+wrong sign, index or transposed operand in the oracle fails one of them.
+
+Method source: "WeightQuantBatchMatmulExperiment 算子深度解析"
+(bjdmk.com.cn/news/4847346), section 4.1, equations 1-11.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from inputs import make_case, pack_int4, workload
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+# 0.5 / (7.49 * 14.98^2): the largest value the dropped fourth digit can
+# carry, relative to A_max, after three residual steps (eq. 2-7).
+TRUNC = 0.5 / (7.49 * 14.98 * 14.98)
+
+
+# ---------------------------------------------------------------- binary16
+
+def test_half_to_double_all_bit_patterns():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    h = bits.view(np.float16)
+    ours = oracle.half_to_double(h)
+    ref = h.astype(np.float64)
+    finite = np.isfinite(ref)
+    assert np.array_equal(ours[finite], ref[finite])
+    assert np.array_equal(np.isnan(ours), np.isnan(ref))
+    inf = np.isinf(ref)
+    assert np.array_equal(ours[inf], ref[inf])
+
+
+def test_double_to_half_matches_numpy_rounding():
+    rng = np.random.default_rng(1)
+    v = np.concatenate([
+        rng.standard_normal(20000) * 10.0 ** rng.integers(-9, 5, 20000),
+        # exact ties between neighbouring halves, both parities
+        (np.arange(4096, dtype=np.float64) + 0.5) * 2.0 ** -24,
+        (np.arange(1024, 2048, dtype=np.float64) + 0.5) * 2.0 ** -10,
+        np.array([65504.0, 65519.99, 65520.0, 1e6, -0.0, 0.0, 6e-8, 2.9e-8, 3.0e-8]),
+    ])
+    ours = oracle.double_to_half(v).view(np.uint16)
+    ref = v.astype(np.float16).view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+# ---------------------------------------------------------------- int4 decode
+
+def test_unpack_nibble_order_and_sign_literal():
+    # byte 0x9F: low nibble 0xF -> W[0] = -1, high nibble 0x9 -> W[1] = -7
+    # byte 0x70: low 0x0 -> 0, high 0x7 -> 7 ; byte 0x08: low 0x8 -> -8, high 0
+    wp = np.array([[0x9F, 0x70, 0x08]], dtype=np.uint8)
+    w = oracle.unpack_w(wp, 2, 3)
+    assert w.tolist() == [[-1, 0, -8], [-7, 7, 0]]
+
+
+def test_unpack_every_byte():
+    b = np.arange(256, dtype=np.uint8).reshape(1, 256)
+    w = oracle.unpack_w(b, 2, 256)
+    lo = np.arange(256) & 15
+    hi = np.arange(256) >> 4
+    assert np.array_equal(w[0], np.where(lo >= 8, lo - 16, lo))
+    assert np.array_equal(w[1], np.where(hi >= 8, hi - 16, hi))
+
+
+# ---------------------------------------------------------------- worked example
+
+def _golden():
+    with open(os.path.join(GOLDEN, "msd_worked_example.json")) as f:
+        return json.load(f)
+
+
+@pytest.mark.parametrize("mode", [oracle.MODE_FP32, oracle.MODE_FP64])
+def test_worked_example_digits_and_yint(mode):
+    ex = _golden()
+    g = ex["g"]
+    x = np.array([ex["x"]], dtype=np.float16)
+    w = np.array(ex["w"], dtype=np.int8)
+    amax, a = oracle.msd_expand(x, g, mode)
+    assert amax[0, 0] == ex["amax"]
+    assert a[0, 0].tolist() == ex["A1"]
+    assert a[1, 0].tolist() == ex["A2"]
+    assert a[2, 0].tolist() == ex["A3"]
+    yint = oracle.msd_yint(a, pack_int4(w), w.shape[1], g)
+    assert yint[0, 0, 0].tolist() == ex["Y1"]
+    assert yint[1, 0, 0].tolist() == ex["Y2"]
+    assert yint[2, 0, 0].tolist() == ex["Y3"]
+
+
+def test_worked_example_output():
+    ex = _golden()
+    g = ex["g"]
+    x = np.array([ex["x"]], dtype=np.float16)
+    w = np.array(ex["w"], dtype=np.int8)
+    scale = np.array([ex["scale"]], dtype=np.float16)
+    y = oracle.msd(x, pack_int4(w), scale, g)
+    np.testing.assert_allclose(y[0], ex["y_msd"], rtol=1e-12, atol=0)
+    ye = oracle.dequant(x, pack_int4(w), scale, g)
+    np.testing.assert_allclose(ye[0], ex["y_exact"], rtol=1e-15, atol=0)
+    assert np.all(np.abs(y[0] - ye[0]) <= np.array(ex["truncation_bound"]))
+
+
+# ---------------------------------------------------------------- invariants
+
+def _adversarial_x(rng, M, K, g):
+    x = rng.standard_normal((M, K)).astype(np.float16)
+    x[0] = 0                                  # all-zero groups
+    x[1, :g] = np.float16(3.0)                # all entries equal +A_max
+    x[1, g:2 * g] = np.float16(-0.5)          # all entries equal -A_max
+    x[2] = rng.integers(-3, 4, K).astype(np.float16)     # small integers
+    x[3] *= np.float16(1e-4)                  # tiny values (subnormals)
+    x[4, ::7] *= np.float16(2000)             # big outliers
+    return x
+
+
+@pytest.mark.parametrize("mode", [oracle.MODE_FP32, oracle.MODE_FP64])
+def test_digits_bounded_by_seven(mode):
+    """|tmp1| <= 7.49 and each residual |tmp - round(tmp)| <= 0.5, so after the
+    x14.98 rescale every digit satisfies |A_i| <= 7 (fits symmetric int4)."""
+    rng = np.random.default_rng(7)
+    for g in (32, 64, 128):
+        x = _adversarial_x(rng, 8, 512, g)
+        _, a = oracle.msd_expand(x, g, mode)
+        assert np.abs(a).max() <= 7
+
+
+def test_equal_magnitude_group_digits():
+    """x = +-A_max everywhere: tmp1 = +-7.49 -> A1 = +-7; tmp2 = +-0.49*14.98 =
+    +-7.3402 -> A2 = +-7; tmp3 = +-0.3402*14.98 = +-5.0962 -> A3 = +-5."""
+    x = np.array([[2.0] * 4 + [-2.0] * 4], dtype=np.float16)
+    amax, a = oracle.msd_expand(x, 4)
+    assert amax.tolist() == [[2.0, 2.0]]
+    assert a[:, 0, :4].tolist() == [[7] * 4, [7] * 4, [5] * 4]
+    assert a[:, 0, 4:].tolist() == [[-7] * 4, [-7] * 4, [-5] * 4]
+
+
+def test_zero_group_contributes_nothing():
+    c = make_case(4, 256, 64, 64, seed=3)
+    c.x[1, 64:128] = 0
+    amax, a = oracle.msd_expand(c.x, 64)
+    assert amax[1, 1] == 0 and not a[:, 1, 64:128].any()
+    y = oracle.msd(c.x, c.wp[0], c.scale[0], 64)
+    # zeroing the group's scale changes nothing for row 1
+    s2 = c.scale[0].copy()
+    s2[1] = 0
+    y2 = oracle.msd(c.x, c.wp[0], s2, 64)
+    assert np.array_equal(y[1], y2[1])
+    assert not np.array_equal(y[0], y2[0])
+
+
+@pytest.mark.parametrize("mode", [oracle.MODE_FP32, oracle.MODE_FP64])
+def test_digit_reconstruction(mode):
+    """7.49*x/A_max = A1 + A2/14.98 + A3/14.98^2 + r/14.98^2 with |r| <= 0.5."""
+    rng = np.random.default_rng(11)
+    g = 64
+    x = _adversarial_x(rng, 8, 256, g)
+    amax, a = oracle.msd_expand(x, g, mode)
+    xd = x.astype(np.float64)
+    am = np.repeat(amax, g, axis=1)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        t = np.where(am > 0, 7.49 * xd / am, 0.0)
+    rec = a[0] + a[1] / 14.98 + a[2] / 14.98 ** 2
+    slack = 0.5 / 14.98 ** 2 * (1.0 if mode == oracle.MODE_FP64 else 1.02)
+    assert np.abs(t - rec).max() <= slack + 1e-12
+
+
+# ---------------------------------------------------------------- against exact GEMMs
+
+def _exact_gemm(x, w, scale, g):
+    """fp64 GEMM by numpy (a library primitive, another summation order)."""
+    s = np.repeat(scale.astype(np.float64), g, axis=0)
+    return x.astype(np.float64) @ (s * w.astype(np.float64))
+
+
+def _truncation_bound(amax, w, scale, g):
+    K, N = w.shape
+    G = K // g
+    absw = np.abs(w.astype(np.float64)).reshape(G, g, N).sum(axis=1)      # [G, N]
+    return TRUNC * (amax @ (np.abs(scale.astype(np.float64)) * absw))     # [M, N]
+
+
+@pytest.mark.parametrize("g", [32, 64, 128])
+def test_dequant_oracle_matches_numpy_gemm(g):
+    c = make_case(5, 512, 96, g, seed=20 + g, keep_w=True)
+    y = oracle.dequant(c.x, c.wp[0], c.scale[0], g)
+    ref = _exact_gemm(c.x, c.w[0], c.scale[0], g)
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_dequant_integer_special_case_is_exact():
+    """scale = 1 and small-integer x: the exact GEMM is an integer GEMM."""
+    rng = np.random.default_rng(5)
+    K, N, g = 256, 40, 64
+    xi = rng.integers(-4, 5, (3, K))
+    w = rng.integers(-8, 8, (K, N)).astype(np.int8)
+    y = oracle.dequant(xi.astype(np.float16), pack_int4(w), np.ones((K // g, N), np.float16), g)
+    assert np.array_equal(y, (xi @ w.astype(np.int64)).astype(np.float64))
+
+
+def test_dequant_single_group_dot_product():
+    """g = K, M = 1: one scale per column, a textbook dot product."""
+    rng = np.random.default_rng(9)
+    K, N = 64, 3
+    x = rng.standard_normal((1, K)).astype(np.float16)
+    w = rng.integers(-8, 8, (K, N)).astype(np.int8)
+    s = np.array([[0.5, -0.25, 0.125]], np.float16)
+    y = oracle.dequant(x, pack_int4(w), s, K)
+    for n in range(N):
+        ref = float(s[0, n]) * sum(float(x[0, k]) * int(w[k, n]) for k in range(K))
+        assert abs(y[0, n] - ref) <= 1e-12 * max(1.0, abs(ref))
+
+
+@pytest.mark.parametrize("mode", [oracle.MODE_FP32, oracle.MODE_FP64])
+@pytest.mark.parametrize("g", [32, 64, 128])
+def test_msd_within_truncation_bound_of_exact(mode, g):
+    """The MSD result stays within the decomposition's truncation error of the
+    exact GEMM (binary64 expansion: exactly; binary32: a 2% slack covers the
+    gap between 7.49f/14.98f and 7.49/14.98 and the rounding of tmp)."""
+    c = make_case(6, 512, 80, g, seed=40 + g, keep_w=True)
+    c.x[2, :g] = 0
+    amax, _ = oracle.msd_expand(c.x, g, mode)
+    y = oracle.msd(c.x, c.wp[0], c.scale[0], g, mode)
+    ye = _exact_gemm(c.x, c.w[0], c.scale[0], g)
+    bound = _truncation_bound(amax, c.w[0], c.scale[0], g)
+    slack = 1.0 if mode == oracle.MODE_FP64 else 1.02
+    assert np.all(np.abs(y - ye) <= bound * slack + 1e-12)
+    # and the error is not trivially zero: MSD is an approximation
+    assert np.abs(y - ye).max() > 0
+
+
+def test_msd_yint_matches_integer_gemm():
+    c = make_case(4, 256, 48, 64, seed=77, keep_w=True)
+    amax, a = oracle.msd_expand(c.x, 64)
+    yint = oracle.msd_yint(a, c.wp[0], 48, 64)
+    w = c.w[0].astype(np.int64)
+    for r in range(3):
+        for gi in range(4):
+            ref = a[r].astype(np.int64)[:, gi * 64:(gi + 1) * 64] @ w[gi * 64:(gi + 1) * 64]
+            assert np.array_equal(yint[r, :, gi], ref)
+    # the magnitude bound |Y| <= 7 * 8 * g
+    assert np.abs(yint).max() <= 7 * 8 * 64
+
+
+def test_msd_brute_force_tiny():
+    """Tiny shapes, every weight value: the stored-Y path (eq. 9 then 10-11)
+    equals the fused per-row path, and both meet the truncation bound."""
+    for K, g in ((2, 2), (4, 2), (8, 4), (8, 8)):
+        for N in (1, 3):
+            for seed in range(4):
+                c = make_case(2, K, N, g, seed=1000 + seed, keep_w=True)
+                amax, a = oracle.msd_expand(c.x, g)
+                yint = oracle.msd_yint(a, c.wp[0], N, g)
+                y1 = oracle.msd_combine(yint, amax, c.scale[0], K, g)
+                y2 = oracle.msd(c.x, c.wp[0], c.scale[0], g)
+                assert np.array_equal(y1, y2)
+                ye = _exact_gemm(c.x, c.w[0], c.scale[0], g)
+                bound = _truncation_bound(amax, c.w[0], c.scale[0], g)
+                assert np.all(np.abs(y2 - ye) <= bound * 1.02 + 1e-15)
+    # all 16 weight values in one column
+    w = np.arange(-8, 8, dtype=np.int8).reshape(16, 1)
+    x = np.linspace(-1, 1, 16).astype(np.float16).reshape(1, 16)
+    s = np.array([[0.75]], np.float16)
+    y = oracle.msd(x, pack_int4(w), s, 16)
+    amax, a = oracle.msd_expand(x, 16)
+    ye = _exact_gemm(x, w, s, 16)
+    assert abs(y[0, 0] - ye[0, 0]) <= _truncation_bound(amax, w, s, 16)[0, 0] * 1.02
+
+
+def test_sampled_outputs_match_full():
+    c = make_case(7, 256, 64, 64, seed=5)
+    rows = np.array([6, 0, 3, 3, 6, 1])
+    cols = np.array([63, 0, 17, 2, 5, 40])
+    y = oracle.msd(c.x, c.wp[0], c.scale[0], 64)
+    assert np.array_equal(oracle.msd_at(c.x, c.wp[0], c.scale[0], 64, rows, cols), y[rows, cols])
+    yd = oracle.dequant(c.x, c.wp[0], c.scale[0], 64)
+    assert np.array_equal(oracle.dequant_at(c.x, c.wp[0], c.scale[0], 64, rows, cols),
+                          yd[rows, cols])
+
+
+def test_grouped_oracle_segments():
+    c = make_case(40, 128, 32, 64, seed=9, E=3)
+    c.offsets[:] = [0, 10, 10, 40]          # an empty expert in the middle
+    y = oracle.grouped("dequant", c.x, c.wp, c.scale, c.offsets, 64)
+    assert np.array_equal(y[:10], oracle.dequant(c.x[:10], c.wp[0], c.scale[0], 64))
+    assert np.array_equal(y[10:], oracle.dequant(c.x[10:], c.wp[2], c.scale[2], 64))
+    rows, cols = np.array([0, 9, 10, 39]), np.array([1, 2, 3, 31])
+    assert np.array_equal(oracle.grouped_at("msd", c.x, c.wp, c.scale, c.offsets, 64, rows, cols),
+                          oracle.grouped("msd", c.x, c.wp, c.scale, c.offsets, 64)[rows, cols])
+
+
+def test_workload_table():
+    """The five workloads keep the shapes the benchmark and parity tests use."""
+    assert (workload(0).M, workload(0).K, workload(0).N, workload(0).g) == (16, 256, 256, 64)
+    assert (workload(1).M, workload(1).K, workload(1).N, workload(1).g) == (1, 4096, 4096, 128)
+    assert (workload(2).M, workload(2).N) == (16, 14336)
+    assert (workload(3).M, workload(3).N) == (4096, 4096)
+    assert (workload(4).E, workload(4).M, workload(4).N) == (8, 4096, 14336)
