@@ -1,0 +1,185 @@
+/*
+ * w4a16.h -- C ABI of the B200 (sm_100a) A16W4 per-group weight-quantised
+ * matmul library (libw4a16.so).
+ *
+ *   y[M, N] = x[M, K] . (antiquant_scale (.) W)[K, N]
+ *
+ * with fp16 activations x, signed int4 weights W, one fp16 scale per group
+ * of g consecutive K rows and per column, and an fp16 result y.  This is the
+ * operator of "WeightQuantBatchMatmulExperiment 算子深度解析"
+ * (bjdmk.com.cn/news/4847346), section 4.2 (x float16/ND, weight int4/ND,
+ * antiquant_scale float16/ND, y float16/ND, all 2-D).  Two algorithms compute it:
+ *
+ *   MSD      the multi-step decomposition of section 4.1, equations 1-11:
+ *            per (row, group) A_max = max|x|; three int4 residual digits
+ *            A1..A3 from 7.49*x/A_max with two x14.98 residual steps; three
+ *            exact integer matmuls Y1..Y3 against the int4 weights; combined
+ *            as (Y1/7.49 + Y2/(7.49*14.98) + Y3/(7.49*14.98^2))*A_max*scale
+ *            and accumulated over groups.
+ *   DEQUANT  the direct dequantise-in-register W4A16 GEMM that the pages
+ *            discuss as Marlin ("pwwt.cn/news/2290475", sections 1.6 and 6)
+ *            and QUICK ("briefgpt.xyz/kw/cuda kernels", QUICK abstract):
+ *            W' = fp16(scale * W), y = x . W' with fp32 accumulation.
+ *
+ * Conventions for every entry point
+ *  - Pointers marked "device" are CUDA device pointers owned by the caller;
+ *    pointers marked "host" are host memory owned by the caller.  The
+ *    library allocates no memory and keeps no state between calls.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream).  No entry point synchronises the stream, except
+ *    w4a16_read_status, which says so.
+ *  - Arguments are validated on the host before anything is launched; a
+ *    failed check returns an error status and launches nothing.  No entry
+ *    point throws or aborts.  A failed launch returns W4A16_ERR_CUDA.
+ *  - Device-side waits are bounded.  A wait that expires makes the kernel
+ *    record W4A16_DEVICE_TIMEOUT in the workspace status word and return;
+ *    read it with w4a16_read_status after the stream has drained.
+ *  - Layouts: x row-major [M][K]; y row-major [M][N]; scale row-major
+ *    [K/g][N]; logical weights as bytes [K/2][N] whose byte (i, n) holds
+ *    W[2i][n] in the low nibble and W[2i+1][n] in the high nibble, two's
+ *    complement ("two int4 per byte", section 4.3 of the same page).
+ *  - Shape rules: M >= 0, K > 0, N > 0; N % 8 == 0; g % 32 == 0 and either
+ *    128 % g == 0 (g = 32, 64, 128) or g % 128 == 0; K % g == 0.  x, y,
+ *    scale and packed weights must be 16-byte aligned.  Inputs must be finite.
+ */
+#ifndef W4A16_H
+#define W4A16_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t. */
+typedef struct CUstream_st* w4a16_stream_t;
+
+typedef enum {
+    W4A16_OK = 0,
+    W4A16_ERR_INVALID_ARG = 1,   /* null pointer, bad shape, misalignment     */
+    W4A16_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. g = 96)   */
+    W4A16_ERR_WORKSPACE = 3,     /* workspace missing or smaller than needed  */
+    W4A16_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed      */
+    W4A16_ERR_TIMEOUT = 5        /* a device wait expired (see status word)   */
+} w4a16_status;
+
+/* Operation selector for w4a16_workspace_size and w4a16_grouped_matmul. */
+enum { W4A16_OP_MSD = 0, W4A16_OP_DEQUANT = 1 };
+
+/* Bits of the device status word kept at the start of every workspace. */
+enum { W4A16_DEVICE_TIMEOUT = 1u };
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* w4a16_status_string(w4a16_status s);
+
+/* Bytes of the packed (kernel-layout) weight buffer for a K x N int4 matrix:
+ * ceil(N/128) * ceil(K/128) * 8192.  Equals K*N/2 when K and N are
+ * multiples of 128.  Returns 0 for non-positive sizes. */
+size_t w4a16_packed_bytes(int K, int N);
+
+/* Bytes of workspace a matmul call needs.
+ *   op: W4A16_OP_MSD or W4A16_OP_DEQUANT; M: rows of x (for grouped calls,
+ *   the total token count T); E: 1 for the dense calls, the expert count for
+ *   w4a16_grouped_matmul.  The workspace holds the device status word, the
+ *   split-K partial sums and arrival counters, and (MSD) the expanded
+ *   activations A_int [3][M][K] int8 and A_max [K/g][M] fp32.
+ * The workspace must be zero-filled before its first use; every call leaves
+ * its counters at zero again, so it can be reused by later calls on the same
+ * stream.  Calls that overlap in time must not share a workspace.  After a
+ * call that reported a device timeout, zero it again.
+ * Returns W4A16_ERR_INVALID_ARG / W4A16_ERR_UNSUPPORTED on bad shapes. */
+w4a16_status w4a16_workspace_size(int op, int M, int K, int N, int group_size,
+                                  int E, size_t* bytes);
+
+/* a0: offline weight re-layout (the "Marlin layout" idea of pwwt.cn/news/2290475
+ * section 6.2 and QUICK's offline interleave): logical packed bytes -> the
+ * kernel layout, so each 128-column tile and 128-deep K chunk is one
+ * contiguous 8 KB block that a single bulk copy brings into shared memory.
+ *   w_logical  device, uint8 [K/2][N] (layout above)
+ *   w_packed   device, w4a16_packed_bytes(K, N) bytes, written fully
+ *              (padding columns/rows are written as zero weights)
+ * K must be even and N % 8 == 0 (the matmul shape rules apply when the
+ * packed buffer is used). */
+w4a16_status w4a16_repack(const uint8_t* w_logical, int K, int N, void* w_packed,
+                          w4a16_stream_t stream);
+
+/* MSD variant, equations 1-11 of section 4.1.
+ *   x          device fp16 [M][K]
+ *   w_packed   device, produced by w4a16_repack for (K, N)
+ *   scale      device fp16 [K/g][N]
+ *   y          device fp16 [M][N], fully overwritten (round-to-nearest-even)
+ *   workspace  device, >= w4a16_workspace_size(W4A16_OP_MSD, M, K, N, g, 1)
+ * Step 1-8 (A_max and the residual digits, binary32 arithmetic with the
+ * constants 7.49f and 14.98f) run in one kernel that writes A_int and A_max
+ * to the workspace; steps 9-11 (tcgen05 int8 MMAs with exact int32
+ * accumulators, the combine and the group accumulation in fp32) in a second.
+ * M == 0 is a no-op. */
+w4a16_status w4a16_msd_matmul(const void* x, const void* w_packed, const void* scale,
+                              int M, int K, int N, int group_size, void* y,
+                              void* workspace, size_t workspace_bytes,
+                              w4a16_stream_t stream);
+
+/* Direct dequant variant: W' = fp16(scale * W) in registers, y = x . W' on
+ * the fp16 tensor cores with fp32 accumulation, y rounded to fp16 once.
+ * Arguments as w4a16_msd_matmul (workspace sized for W4A16_OP_DEQUANT). */
+w4a16_status w4a16_dequant_matmul(const void* x, const void* w_packed, const void* scale,
+                                  int M, int K, int N, int group_size, void* y,
+                                  void* workspace, size_t workspace_bytes,
+                                  w4a16_stream_t stream);
+
+/* Grouped-expert (MoE) form: expert e multiplies the contiguous token rows
+ * offsets[e] .. offsets[e+1]-1 of x by its own weights (the dense and MoE
+ * scheduling Humming describes, aihirek.info "Humming ..." article).
+ *   op         W4A16_OP_MSD or W4A16_OP_DEQUANT
+ *   x          device fp16 [T][K], tokens sorted by expert
+ *   w_packed   host array of E device pointers (each from w4a16_repack)
+ *   scale      host array of E device pointers, fp16 [K/g][N] each
+ *   offsets    device int32 [E+1], non-decreasing, offsets[0] = 0,
+ *              offsets[E] = T (empty experts allowed)
+ *   y          device fp16 [T][N], fully overwritten
+ *   workspace  >= w4a16_workspace_size(op, T, K, N, g, E)
+ * 1 <= E <= 64.  Offsets that break the rules above give undefined rows
+ * but no out-of-bounds access: rows are clamped to [0, T). */
+w4a16_status w4a16_grouped_matmul(int op, const void* x, const void* const* w_packed,
+                                  const void* const* scale, const int32_t* offsets,
+                                  int E, int T, int K, int N, int group_size, void* y,
+                                  void* workspace, size_t workspace_bytes,
+                                  w4a16_stream_t stream);
+
+/* Debug window into MSD equation 9: the exact int32 Y1, Y2, Y3 per group
+ * for rows m0..m1-1 and columns n0..n1-1, as accumulated by the tensor
+ * cores, plus A_max.
+ *   yint  device int32 [3][m1-m0][K/g][n1-n0]
+ *   amax  device fp32 [m1-m0][K/g]
+ *   workspace as for w4a16_msd_matmul.
+ * 0 <= m0 < m1 <= M, 0 <= n0 < n1 <= N.  The full tensor is 12*M*N*K/g
+ * bytes, so keep windows small. */
+w4a16_status w4a16_msd_debug_yint(const void* x, const void* w_packed, int M, int K,
+                                  int N, int group_size, int m0, int m1, int n0, int n1,
+                                  int32_t* yint, float* amax, void* workspace,
+                                  size_t workspace_bytes, w4a16_stream_t stream);
+
+/* Copy the device status word at the start of `workspace` into *status
+ * (0 = no device error; W4A16_DEVICE_TIMEOUT bit = a bounded wait expired).
+ * SYNCHRONISES `stream`.  Returns W4A16_ERR_TIMEOUT when the timeout bit is
+ * set, W4A16_OK otherwise. */
+w4a16_status w4a16_read_status(const void* workspace, w4a16_stream_t stream,
+                               uint32_t* status);
+
+/* Set the bound on every device-side wait, in nanoseconds of GPU global
+ * time (default 2e9).  Applies to launches made after the call, process-wide. */
+void w4a16_set_wait_timeout_ns(uint64_t ns);
+
+/* Launch a self-test kernel whose single wait is on a barrier that nothing
+ * completes, bounded by `timeout_ns`; it must record W4A16_DEVICE_TIMEOUT in
+ * the workspace status word and return.  Used to test the timeout path
+ * without hanging a GPU.  workspace: device, >= 256 bytes. */
+w4a16_status w4a16_selftest_wait_timeout(void* workspace, uint64_t timeout_ns,
+                                         w4a16_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A16_H */

@@ -1,0 +1,115 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/w4a16.h declares, and rejects bad arguments
+before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w4a16.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(w4a16_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from weight_only_int4_a16w4_b200 import build
+    build.build()
+    import weight_only_int4_a16w4_b200 as w4
+    return w4
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for n in ("w4a16_repack", "w4a16_msd_matmul", "w4a16_dequant_matmul", "w4a16_grouped_matmul",
+              "w4a16_msd_debug_yint", "w4a16_workspace_size", "w4a16_packed_bytes"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    so = ctypes.CDLL(lib.LIB_PATH)
+    for name in _declared_functions():
+        assert hasattr(so, name), name
+        # the binding exposes the same names
+        assert hasattr(lib, name), name
+
+
+def test_packed_bytes(lib):
+    assert lib.w4a16_packed_bytes(4096, 4096) == 4096 * 4096 // 2
+    assert lib.w4a16_packed_bytes(4096, 14336) == 4096 * 14336 // 2
+    assert lib.w4a16_packed_bytes(192, 136) == 2 * 2 * 8192       # padded to 128 x 128 tiles
+    assert lib.w4a16_packed_bytes(0, 8) == 0
+
+
+def test_workspace_sizes(lib):
+    msd = lib.w4a16_workspace_size(lib.OP_MSD, 16, 4096, 14336, 128)
+    deq = lib.w4a16_workspace_size(lib.OP_DEQUANT, 16, 4096, 14336, 128)
+    # MSD holds A_int (3*M*K bytes) and A_max (K/g*M floats) on top of what DEQUANT needs
+    assert msd - deq >= 3 * 16 * 4096 + 32 * 16 * 4
+    assert lib.w4a16_workspace_size(lib.OP_DEQUANT, 0, 256, 256, 64) >= 256
+    assert lib.w4a16_workspace_size(lib.OP_MSD, 4096, 4096, 14336, 128, E=8) >= 3 * 4096 * 4096
+
+
+@pytest.mark.parametrize("args,code", [
+    ((0, 16, 4096, 4100, 128), 1),      # N % 8 != 0
+    ((0, 16, 4000, 4096, 128), 1),      # K % g != 0
+    ((0, 16, 3840, 4096, 96), 2),       # g = 96 unsupported
+    ((0, -1, 4096, 4096, 128), 1),      # negative M
+    ((0, 16, 4096, 4096, 1024), 2),     # MSD group larger than 512
+    ((7, 16, 4096, 4096, 128), 1),      # bad op
+])
+def test_workspace_size_rejects(lib, args, code):
+    with pytest.raises(lib.W4A16Error) as e:
+        lib.w4a16_workspace_size(*args)
+    assert e.value.code == code
+
+
+def test_matmul_rejects_before_launch(lib):
+    fake = 1 << 40                       # 16-byte aligned, never dereferenced
+    for fn in (lib.w4a16_msd_matmul, lib.w4a16_dequant_matmul):
+        with pytest.raises(lib.W4A16Error) as e:     # null x
+            fn(None, fake, fake, 16, 256, 256, 64, fake, fake, 1 << 20, stream=0)
+        assert e.value.code == 1
+        with pytest.raises(lib.W4A16Error) as e:     # misaligned y
+            fn(fake, fake, fake, 16, 256, 256, 64, fake + 2, fake, 1 << 20, stream=0)
+        assert e.value.code == 1
+        with pytest.raises(lib.W4A16Error) as e:     # workspace too small
+            fn(fake, fake, fake, 16, 256, 256, 64, fake, fake, 16, stream=0)
+        assert e.value.code == 3
+        with pytest.raises(lib.W4A16Error) as e:     # unsupported group
+            fn(fake, fake, fake, 16, 288, 256, 96, fake, fake, 1 << 20, stream=0)
+        assert e.value.code == 2
+    # M == 0 is a no-op that touches nothing
+    lib.w4a16_dequant_matmul(None, None, None, 0, 256, 256, 64, None, None, 0, stream=0)
+
+
+def test_grouped_and_debug_reject(lib):
+    fake = 1 << 40
+    with pytest.raises(lib.W4A16Error) as e:         # too many experts
+        lib.w4a16_grouped_matmul(0, fake, [fake] * 65, [fake] * 65, fake, 65, 64, 256, 256, 64, fake, fake,
+                                 1 << 30, stream=0)
+    assert e.value.code == 1
+    with pytest.raises(lib.W4A16Error) as e:         # null expert weight
+        lib.w4a16_grouped_matmul(1, fake, [fake, None], [fake, fake], fake, 2, 64, 256, 256, 64, fake, fake,
+                                 1 << 30, stream=0)
+    assert e.value.code == 1
+    with pytest.raises(lib.W4A16Error) as e:         # empty debug window
+        lib.w4a16_msd_debug_yint(fake, fake, 16, 256, 256, 64, 3, 3, 0, 8, fake, fake, fake, 1 << 20,
+                                 stream=0)
+    assert e.value.code == 1
+
+
+def test_repack_rejects(lib):
+    fake = 1 << 40
+    with pytest.raises(lib.W4A16Error):
+        lib.w4a16_repack(fake, 255, 256, fake, stream=0)     # odd K
+    with pytest.raises(lib.W4A16Error):
+        lib.w4a16_repack(fake, 256, 250, fake, stream=0)     # N % 8
+    with pytest.raises(lib.W4A16Error):
+        lib.w4a16_repack(fake, 256, 256, fake + 8, stream=0)  # misaligned output

@@ -1,0 +1,279 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle on
+the same seeded inputs.
+
+Bars (from the method's acceptance rules):
+  * MSD equation 9: the per-group int32 Y1, Y2, Y3 (debug window) and A_max
+    are bit-exact against the oracle's.
+  * MSD y: |y - y_oracle| <= 2e-3 * max|y_oracle| + 1e-3, y_oracle the
+    binary64 result of equations 1-11.
+  * DEQUANT y: ||y - y_exact||_F / ||y_exact||_F <= 1e-3 against the exact
+    binary64 GEMM.
+Full-size workloads are checked on sampled outputs the oracle computes one
+by one, in the same launch configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from inputs import make_case, make_workload, pack_int4
+
+pytestmark = pytest.mark.gpu
+
+MSD_REL, MSD_ABS = 2e-3, 1e-3
+DEQ_REL_F = 1e-3
+
+
+def _t():
+    import torch
+    return torch
+
+
+def upload(w4, c):
+    torch = _t()
+    dev = {"x": torch.from_numpy(c.x).cuda()}
+    dev["wp"] = [w4.repack(torch.from_numpy(wp).cuda(), c.K, c.N) for wp in c.wp]
+    dev["scale"] = [torch.from_numpy(s).cuda() for s in c.scale]
+    if c.offsets is not None:
+        dev["offsets"] = torch.from_numpy(c.offsets).cuda()
+    return dev
+
+
+def run_dense(w4, op, c, dev, ws=None):
+    torch = _t()
+    y = torch.full((c.M, c.N), float("nan"), dtype=torch.float16, device="cuda")
+    if ws is None:
+        ws = w4.alloc_workspace(op, c.M, c.K, c.N, c.g)
+    fn = w4.w4a16_msd_matmul if op == w4.OP_MSD else w4.w4a16_dequant_matmul
+    fn(dev["x"], dev["wp"][0], dev["scale"][0], c.M, c.K, c.N, c.g, y, ws)
+    torch.cuda.synchronize()
+    assert w4.w4a16_read_status(ws) == 0
+    return y.cpu().numpy().astype(np.float64)
+
+
+def run_grouped(w4, op, c, dev):
+    torch = _t()
+    T = c.M
+    y = torch.full((T, c.N), float("nan"), dtype=torch.float16, device="cuda")
+    ws = w4.alloc_workspace(op, T, c.K, c.N, c.g, E=c.E)
+    w4.w4a16_grouped_matmul(op, dev["x"], dev["wp"], dev["scale"], dev["offsets"], c.E, T, c.K, c.N, c.g, y, ws)
+    torch.cuda.synchronize()
+    assert w4.w4a16_read_status(ws) == 0
+    return y.cpu().numpy().astype(np.float64)
+
+
+def assert_msd_close(y, ref, what=""):
+    assert np.all(np.isfinite(y)), f"{what}: non-finite output"
+    tol = MSD_REL * np.abs(ref).max() + MSD_ABS
+    err = np.abs(y - ref)
+    i = np.unravel_index(np.argmax(err), err.shape)
+    assert err.max() <= tol, f"{what}: max err {err.max():.3e} at {i} (gpu {y[i]}, oracle {ref[i]}), tol {tol:.3e}"
+
+
+def assert_deq_close(y, ref, what=""):
+    assert np.all(np.isfinite(y)), f"{what}: non-finite output"
+    rel = np.linalg.norm(y - ref) / max(np.linalg.norm(ref), 1e-300)
+    assert rel <= DEQ_REL_F, f"{what}: relative Frobenius error {rel:.3e}"
+
+
+def debug_yint(w4, c, dev, m0, m1, n0, n1):
+    torch = _t()
+    G = c.K // c.g
+    yint = torch.full((3, m1 - m0, G, n1 - n0), -12345, dtype=torch.int32, device="cuda")
+    amax = torch.full((m1 - m0, G), -1.0, dtype=torch.float32, device="cuda")
+    ws = w4.alloc_workspace(w4.OP_MSD, c.M, c.K, c.N, c.g)
+    w4.w4a16_msd_debug_yint(dev["x"], dev["wp"][0], c.M, c.K, c.N, c.g, m0, m1, n0, n1, yint, amax, ws)
+    torch.cuda.synchronize()
+    assert w4.w4a16_read_status(ws) == 0
+    return yint.cpu().numpy(), amax.cpu().numpy()
+
+
+def check_yint(w4, c, dev, m0, m1, n0, n1):
+    yint, amax = debug_yint(w4, c, dev, m0, m1, n0, n1)
+    ref_amax, a = oracle.msd_expand(c.x[m0:m1], c.g)
+    ref = oracle.msd_yint(a, np.ascontiguousarray(c.wp[0][:, n0:n1]), n1 - n0, c.g)
+    assert np.array_equal(amax.astype(np.float64), ref_amax), "A_max differs"
+    bad = np.argwhere(yint.astype(np.int64) != ref)
+    assert bad.size == 0, f"{len(bad)} Y_int mismatches, first at {bad[0]}: gpu {yint[tuple(bad[0])]} " \
+                          f"oracle {ref[tuple(bad[0])]}"
+
+
+# ---------------------------------------------------------------- failure path
+
+def test_bounded_wait_reports_timeout(cuda_lib):
+    torch = _t()
+    w4 = cuda_lib
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    w4.w4a16_selftest_wait_timeout(ws, 2_000_000)       # 2 ms on a barrier nothing completes
+    assert w4.w4a16_read_status(ws) == w4.DEVICE_TIMEOUT
+    # the context is still usable
+    c = make_case(16, 256, 256, 64, seed=3)
+    dev = upload(w4, c)
+    assert_deq_close(run_dense(w4, w4.OP_DEQUANT, c, dev), oracle.dequant(c.x, c.wp[0], c.scale[0], 64))
+
+
+# ---------------------------------------------------------------- small shapes, full comparison
+
+SMALL = [
+    # (M, K, N, g)                       what it covers
+    (16, 256, 256, 64),                  # the 16x256x256 workload shape
+    (1, 256, 128, 128),                  # one row, one tile
+    (5, 384, 136, 64),                   # ragged N (136 = 128 + 8), 3 K chunks
+    (16, 192, 256, 64),                  # K not a multiple of 128
+    (3, 512, 256, 256),                  # group spanning two K chunks
+    (9, 512, 384, 32),                   # four groups per K chunk
+    (17, 256, 264, 128),                 # first M above the decode tile
+    (70, 512, 256, 64),                  # several token tiles, ragged tail
+    (130, 384, 520, 128),                # ragged in every dimension
+]
+
+
+@pytest.mark.parametrize("M,K,N,g", SMALL)
+def test_msd_small(cuda_lib, M, K, N, g):
+    w4 = cuda_lib
+    c = make_case(M, K, N, g, seed=M * 7919 + K * 31 + N + g)
+    if M > 3:
+        c.x[3, :g] = 0                   # an all-zero group
+    dev = upload(w4, c)
+    y = run_dense(w4, w4.OP_MSD, c, dev)
+    assert_msd_close(y, oracle.msd(c.x, c.wp[0], c.scale[0], g), f"msd {M}x{K}x{N} g{g}")
+
+
+@pytest.mark.parametrize("M,K,N,g", SMALL)
+def test_dequant_small(cuda_lib, M, K, N, g):
+    w4 = cuda_lib
+    c = make_case(M, K, N, g, seed=M * 7919 + K * 31 + N + g + 1)
+    dev = upload(w4, c)
+    y = run_dense(w4, w4.OP_DEQUANT, c, dev)
+    assert_deq_close(y, oracle.dequant(c.x, c.wp[0], c.scale[0], g), f"dequant {M}x{K}x{N} g{g}")
+
+
+@pytest.mark.parametrize("M,K,N,g", [(16, 256, 256, 64), (5, 384, 136, 64), (3, 512, 256, 256),
+                                     (9, 512, 384, 32), (70, 512, 256, 64)])
+def test_msd_yint_bit_exact(cuda_lib, M, K, N, g):
+    w4 = cuda_lib
+    c = make_case(M, K, N, g, seed=99 + M + g)
+    c.x[0, :g] = np.float16(-2.5)        # every entry equals -A_max
+    if M > 2:
+        c.x[2] *= np.float16(1e-4)       # tiny values
+    dev = upload(w4, c)
+    check_yint(w4, c, dev, 0, M, 0, N)
+
+
+def test_page_example_distributions(cuda_lib):
+    """The page's own example distributions (x, scale ~ U[-3,3], w in [-7,7]),
+    at a reduced K so the full oracle is quick; negative scales included."""
+    from inputs import page_example
+    w4 = cuda_lib
+    c = page_example(M=4, K=1024, N=1536)
+    dev = upload(w4, c)
+    assert_msd_close(run_dense(w4, w4.OP_MSD, c, dev), oracle.msd(c.x, c.wp[0], c.scale[0], c.g), "msd")
+    assert_deq_close(run_dense(w4, w4.OP_DEQUANT, c, dev), oracle.dequant(c.x, c.wp[0], c.scale[0], c.g),
+                     "dequant")
+
+
+def test_zero_rows_is_noop(cuda_lib):
+    torch = _t()
+    w4 = cuda_lib
+    y = torch.zeros(4, dtype=torch.float16, device="cuda")
+    w4.w4a16_msd_matmul(None, None, None, 0, 256, 256, 64, y, None, 0)
+    w4.w4a16_dequant_matmul(None, None, None, 0, 256, 256, 64, y, None, 0)
+    torch.cuda.synchronize()
+    assert not y.any()
+
+
+def test_repeat_calls_are_deterministic(cuda_lib):
+    """Split-K counters reset themselves; the ordered reduction gives the
+    same bits on every call."""
+    torch = _t()
+    w4 = cuda_lib
+    c = make_case(16, 2048, 1024, 128, seed=1234)
+    dev = upload(w4, c)
+    for op in (w4.OP_MSD, w4.OP_DEQUANT):
+        ws = w4.alloc_workspace(op, c.M, c.K, c.N, c.g)
+        ys = [run_dense(w4, op, c, dev, ws) for _ in range(3)]
+        assert np.array_equal(ys[0], ys[1]) and np.array_equal(ys[1], ys[2])
+    torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------- grouped experts
+
+def test_grouped_small_with_empty_experts(cuda_lib):
+    w4 = cuda_lib
+    c = make_case(150, 256, 264, 64, seed=4242, E=5)
+    c.offsets[:] = [0, 40, 40, 41, 150, 150]         # empty, one-token and empty-last experts
+    dev = upload(w4, c)
+    ref_m = oracle.grouped("msd", c.x, c.wp, c.scale, c.offsets, c.g)
+    ref_d = oracle.grouped("dequant", c.x, c.wp, c.scale, c.offsets, c.g)
+    assert_msd_close(run_grouped(w4, w4.OP_MSD, c, dev), ref_m, "grouped msd")
+    assert_deq_close(run_grouped(w4, w4.OP_DEQUANT, c, dev), ref_d, "grouped dequant")
+
+
+# ---------------------------------------------------------------- full-size workloads
+
+def _samples(rng, M, N, count):
+    return rng.integers(0, M, count), rng.integers(0, N, count)
+
+
+def test_workload_msd_small_full(cuda_lib):
+    """16 x 256 x 256, g = 64, with the forced all-zero group."""
+    w4 = cuda_lib
+    c = make_workload(0)
+    dev = upload(w4, c)
+    assert_msd_close(run_dense(w4, w4.OP_MSD, c, dev), oracle.msd(c.x, c.wp[0], c.scale[0], c.g), "msd")
+    assert_deq_close(run_dense(w4, w4.OP_DEQUANT, c, dev), oracle.dequant(c.x, c.wp[0], c.scale[0], c.g),
+                     "dequant")
+    check_yint(w4, c, dev, 0, 16, 0, 256)
+
+
+def test_workload_decode_m1_full(cuda_lib):
+    """1 x 4096 x 4096, g = 128: every output checked."""
+    w4 = cuda_lib
+    c = make_workload(1)
+    dev = upload(w4, c)
+    assert_msd_close(run_dense(w4, w4.OP_MSD, c, dev), oracle.msd(c.x, c.wp[0], c.scale[0], c.g), "msd")
+    assert_deq_close(run_dense(w4, w4.OP_DEQUANT, c, dev), oracle.dequant(c.x, c.wp[0], c.scale[0], c.g),
+                     "dequant")
+    check_yint(w4, c, dev, 0, 1, 0, 512)
+
+
+def test_workload_decode_m16_sampled(cuda_lib):
+    """16 x 4096 x 14336, g = 128: 2048 sampled outputs plus a Y_int window."""
+    w4 = cuda_lib
+    c = make_workload(2)
+    dev = upload(w4, c)
+    rng = np.random.default_rng(2)
+    rows, cols = _samples(rng, c.M, c.N, 2048)
+    y = run_dense(w4, w4.OP_MSD, c, dev)
+    assert_msd_close(y[rows, cols], oracle.msd_at(c.x, c.wp[0], c.scale[0], c.g, rows, cols), "msd")
+    y = run_dense(w4, w4.OP_DEQUANT, c, dev)
+    assert_deq_close(y[rows, cols], oracle.dequant_at(c.x, c.wp[0], c.scale[0], c.g, rows, cols), "dequant")
+    check_yint(w4, c, dev, 0, 16, 14336 - 136, 14336)
+
+
+def test_workload_prefill_sampled(cuda_lib):
+    """4096 x 4096 x 4096, g = 128: 2048 sampled outputs plus a Y_int window."""
+    w4 = cuda_lib
+    c = make_workload(3)
+    dev = upload(w4, c)
+    rng = np.random.default_rng(3)
+    rows, cols = _samples(rng, c.M, c.N, 2048)
+    y = run_dense(w4, w4.OP_MSD, c, dev)
+    assert_msd_close(y[rows, cols], oracle.msd_at(c.x, c.wp[0], c.scale[0], c.g, rows, cols), "msd")
+    y = run_dense(w4, w4.OP_DEQUANT, c, dev)
+    assert_deq_close(y[rows, cols], oracle.dequant_at(c.x, c.wp[0], c.scale[0], c.g, rows, cols), "dequant")
+    check_yint(w4, c, dev, 4000, 4096, 4096 - 40, 4096)
+
+
+def test_workload_moe_sampled(cuda_lib):
+    """E = 8, T = 4096, K = 4096, N = 14336: 2048 sampled outputs."""
+    w4 = cuda_lib
+    c = make_workload(4)
+    dev = upload(w4, c)
+    rng = np.random.default_rng(4)
+    rows, cols = _samples(rng, c.M, c.N, 2048)
+    y = run_grouped(w4, w4.OP_MSD, c, dev)
+    assert_msd_close(y[rows, cols], oracle.grouped_at("msd", c.x, c.wp, c.scale, c.offsets, c.g, rows, cols),
+                     "moe msd")
+    y = run_grouped(w4, w4.OP_DEQUANT, c, dev)
+    assert_deq_close(y[rows, cols],
+                     oracle.grouped_at("dequant", c.x, c.wp, c.scale, c.offsets, c.g, rows, cols), "moe dequant")

@@ -1,0 +1,441 @@
+// w4a16_api.cu -- host side of libw4a16.so: argument validation, workspace
+// layout, TMA descriptors, launch-shape choice and the extern "C" entry
+// points declared in include/w4a16.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/w4a16.h"
+#include "w4a16_kernels.cuh"
+
+using namespace w4a16;
+
+namespace {
+
+std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
+
+constexpr size_t kHeaderBytes = 256;   // device status word + padding
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+bool group_ok(int g)
+{
+    if (g <= 0 || g % 32) return false;
+    return (g <= kKC) ? (kKC % g == 0) : (g % kKC == 0);
+}
+
+// ---------------------------------------------------------------- device facts
+
+int sm_count()
+{
+    static std::mutex mu;
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cached[dev] == 0) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+        cached[dev] = v;
+    }
+    return cached[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D K-major tensor map, 128-byte swizzle, box = (box_k, box_rows).
+bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes, int K, int rows,
+              int box_k, int box_rows)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * elem_bytes};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(box_k), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- launch shapes
+
+// Kernel instances:  (variant, token tile, load stages, A stages, CTAs/SM)
+//   decode (M <= 16):  MSD <kMsd,16,7,4,2>   DEQUANT <kDeq,16,8,2,2>
+//   larger M:          MSD <kMsd,64,4,4,1>   DEQUANT <kDeq,128,2,2,2>
+struct Shape {
+    int TT;
+    int splits;
+    int unit;
+    int t_slots;
+    int n_tiles;
+    int kchunks;
+};
+
+bool small_tile(int op, int M) { (void)op; return M <= 16; }
+
+int tile_tokens(int op, int M)
+{
+    if (small_tile(op, M)) return 16;
+    return op == W4A16_OP_MSD ? 64 : 128;
+}
+
+// Split-K factor for a dense call: spread (column tiles x token tiles) work
+// over every SM when there are fewer tiles than SMs, minimising the number
+// of chunk-steps on the busiest SM (2 resident CTAs per SM for the decode tile).
+int choose_splits(int tiles, int units, int resident)
+{
+    const int slots = std::max(1, sm_count() * resident);
+    if (tiles >= sm_count() || units <= 1) return 1;
+    long best_cost = -1;
+    int best = 1;
+    for (int s = 1; s <= units; ++s) {
+        const long ctas = static_cast<long>(tiles) * s;
+        const long waves = (ctas + slots - 1) / slots;
+        const long cost = waves * ((units + s - 1) / s);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = s;
+        }
+    }
+    return best;
+}
+
+Shape dense_shape(int op, int M, int K, int N, int g)
+{
+    Shape s;
+    s.TT = tile_tokens(op, M);
+    s.kchunks = cdiv(K, kKC);
+    s.n_tiles = cdiv(N, kBN);
+    s.t_slots = std::max(1, cdiv(M, s.TT));
+    s.unit = std::max(1, g / kKC);
+    const int units = cdiv(s.kchunks, s.unit);
+    s.splits = small_tile(op, M) ? choose_splits(s.n_tiles * s.t_slots, units, 2) : 1;
+    return s;
+}
+
+Shape grouped_shape(int op, int T, int K, int N, int g, int E)
+{
+    Shape s;
+    s.TT = tile_tokens(op, 1 << 20);
+    s.kchunks = cdiv(K, kKC);
+    s.n_tiles = cdiv(N, kBN);
+    s.t_slots = std::max(1, cdiv(T, s.TT) + E);
+    s.unit = std::max(1, g / kKC);
+    s.splits = 1;
+    return s;
+}
+
+struct WsLayout {
+    size_t counters = 0, partial = 0, xq = 0, amax = 0, total = 0;
+};
+
+WsLayout ws_layout(int op, const Shape& s, int M, int K, int N, int g)
+{
+    WsLayout L;
+    size_t off = kHeaderBytes;
+    if (s.splits > 1) {
+        L.counters = off;
+        off += align256(static_cast<size_t>(s.t_slots) * s.n_tiles * 4);
+        L.partial = off;
+        off += align256(static_cast<size_t>(s.splits) * M * N * 4);
+    }
+    if (op == W4A16_OP_MSD) {
+        L.xq = off;
+        off += align256(static_cast<size_t>(3) * M * K);
+        L.amax = off;
+        off += align256(static_cast<size_t>(K / g) * M * 4);
+    }
+    L.total = off;
+    return L;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+w4a16_status check_shape(int M, int K, int N, int g)
+{
+    if (M < 0 || K <= 0 || N <= 0 || g <= 0) return W4A16_ERR_INVALID_ARG;
+    if (N % 8 || K % g) return W4A16_ERR_INVALID_ARG;
+    if (!group_ok(g)) return W4A16_ERR_UNSUPPORTED;
+    return W4A16_OK;
+}
+
+// ---------------------------------------------------------------- kernel launch
+
+template <int VAR, int TT, int LS, int AS, int MINB>
+w4a16_status launch_gemm(const CUtensorMap& map, const GemmParams& P, dim3 grid, cudaStream_t stream)
+{
+    using C = GemmCfg<VAR, TT, LS, AS>;
+    auto kern = gemm_kernel<VAR, TT, LS, AS, MINB>;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [&] {
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    });
+    if (attr_err != cudaSuccess) return W4A16_ERR_CUDA;
+    kern<<<grid, kThreads, C::kSmem, stream>>>(map, P);
+    return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+}
+
+w4a16_status launch_for(int op, int TT, const CUtensorMap& map, const GemmParams& P, dim3 grid, cudaStream_t s)
+{
+    if (op == W4A16_OP_MSD) {
+        if (TT == 16) return launch_gemm<kMsd, 16, 7, 4, 2>(map, P, grid, s);
+        return launch_gemm<kMsd, 64, 4, 4, 1>(map, P, grid, s);
+    }
+    if (TT == 16) return launch_gemm<kDeq, 16, 8, 2, 2>(map, P, grid, s);
+    return launch_gemm<kDeq, 128, 2, 2, 2>(map, P, grid, s);
+}
+
+w4a16_status launch_expand(const void* x, int M, int K, int g, int8_t* xq, float* amax, cudaStream_t s)
+{
+    const long long warps = static_cast<long long>(M) * (K / g);
+    const int blocks = static_cast<int>((warps + 7) / 8);
+    const __half* xh = static_cast<const __half*>(x);
+    switch (g / 32) {
+        case 1: expand_kernel<1><<<blocks, 256, 0, s>>>(xh, M, K, g, xq, amax); break;
+        case 2: expand_kernel<2><<<blocks, 256, 0, s>>>(xh, M, K, g, xq, amax); break;
+        case 4: expand_kernel<4><<<blocks, 256, 0, s>>>(xh, M, K, g, xq, amax); break;
+        case 8: expand_kernel<8><<<blocks, 256, 0, s>>>(xh, M, K, g, xq, amax); break;
+        case 16: expand_kernel<16><<<blocks, 256, 0, s>>>(xh, M, K, g, xq, amax); break;
+        default: return W4A16_ERR_UNSUPPORTED;
+    }
+    return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+}
+
+void base_params(GemmParams& P, int M, int K, int N, int g, const Shape& s, void* ws)
+{
+    std::memset(&P, 0, sizeof(P));
+    P.M = M;
+    P.K = K;
+    P.N = N;
+    P.g = g;
+    P.G = K / g;
+    P.kchunks = s.kchunks;
+    P.n_tiles = s.n_tiles;
+    P.t_slots = s.t_slots;
+    P.splits = s.splits;
+    P.unit = s.unit;
+    P.E = 1;
+    P.status = static_cast<uint32_t*>(ws);
+    P.timeout_ns = g_timeout_ns.load();
+    P.write_y = 1;
+}
+
+// Shared body of the dense MSD / DEQUANT calls and the debug window.
+w4a16_status dense_matmul(int op, const void* x, const void* w_packed, const void* scale, int M, int K, int N,
+                          int g, void* y, void* ws, size_t ws_bytes, cudaStream_t stream, int32_t* dbg_yint,
+                          float* dbg_amax, int m0, int m1, int n0, int n1)
+{
+    w4a16_status st = check_shape(M, K, N, g);
+    if (st != W4A16_OK) return st;
+    if (op == W4A16_OP_MSD && g > kMaxGroupMsd) return W4A16_ERR_UNSUPPORTED;
+    if (M == 0) return W4A16_OK;
+    const bool debug = dbg_yint != nullptr;
+    if (!x || !w_packed || (!scale && !debug) || (!y && !debug) || !ws) return W4A16_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_packed) || (scale && !aligned16(scale)) || (y && !aligned16(y)) ||
+        !aligned16(ws))
+        return W4A16_ERR_INVALID_ARG;
+    Shape s = dense_shape(op, M, K, N, g);
+    const WsLayout full = ws_layout(op, s, M, K, N, g);
+    if (debug) s.splits = 1;
+    const WsLayout L = ws_layout(op, s, M, K, N, g);
+    if (ws_bytes < full.total) return W4A16_ERR_WORKSPACE;
+
+    GemmParams P;
+    base_params(P, M, K, N, g, s, ws);
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    P.w[0] = static_cast<const uint8_t*>(w_packed);
+    P.scale[0] = static_cast<const __half*>(scale);
+    P.y = static_cast<__half*>(y);
+    if (s.splits > 1) {
+        P.counters = reinterpret_cast<uint32_t*>(wsb + L.counters);
+        P.partial = reinterpret_cast<float*>(wsb + L.partial);
+    }
+    if (debug) {
+        P.write_y = 0;
+        P.dbg_yint = dbg_yint;
+        P.dbg_amax = dbg_amax;
+        P.dbg_m0 = m0;
+        P.dbg_m1 = m1;
+        P.dbg_n0 = n0;
+        P.dbg_n1 = n1;
+    }
+    CUtensorMap map;
+    if (op == W4A16_OP_MSD) {
+        int8_t* xq = reinterpret_cast<int8_t*>(wsb + L.xq);
+        float* amax = reinterpret_cast<float*>(wsb + L.amax);
+        st = launch_expand(x, M, K, g, xq, amax, stream);
+        if (st != W4A16_OK) return st;
+        P.amax = amax;
+        if (!make_map(&map, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, 3 * M, kKC, s.TT)) return W4A16_ERR_CUDA;
+    } else {
+        if (!make_map(&map, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K, M, 64, s.TT)) return W4A16_ERR_CUDA;
+    }
+    dim3 grid(s.n_tiles, s.splits, s.t_slots);
+    return launch_for(op, s.TT, map, P, grid, stream);
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+
+extern "C" {
+
+const char* w4a16_status_string(w4a16_status s)
+{
+    switch (s) {
+        case W4A16_OK: return "ok";
+        case W4A16_ERR_INVALID_ARG: return "invalid argument";
+        case W4A16_ERR_UNSUPPORTED: return "unsupported shape or group size";
+        case W4A16_ERR_WORKSPACE: return "workspace missing or too small";
+        case W4A16_ERR_CUDA: return "CUDA error";
+        case W4A16_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+size_t w4a16_packed_bytes(int K, int N)
+{
+    if (K <= 0 || N <= 0) return 0;
+    return static_cast<size_t>(cdiv(N, kBN)) * cdiv(K, kKC) * kWStage;
+}
+
+w4a16_status w4a16_workspace_size(int op, int M, int K, int N, int group_size, int E, size_t* bytes)
+{
+    if (!bytes) return W4A16_ERR_INVALID_ARG;
+    if (op != W4A16_OP_MSD && op != W4A16_OP_DEQUANT) return W4A16_ERR_INVALID_ARG;
+    if (E < 1 || E > kMaxExperts) return W4A16_ERR_INVALID_ARG;
+    w4a16_status st = check_shape(M, K, N, group_size);
+    if (st != W4A16_OK) return st;
+    if (op == W4A16_OP_MSD && group_size > kMaxGroupMsd) return W4A16_ERR_UNSUPPORTED;
+    const Shape s = (E == 1) ? dense_shape(op, M, K, N, group_size) : grouped_shape(op, M, K, N, group_size, E);
+    *bytes = ws_layout(op, s, M, K, N, group_size).total;
+    return W4A16_OK;
+}
+
+w4a16_status w4a16_repack(const uint8_t* w_logical, int K, int N, void* w_packed, w4a16_stream_t stream)
+{
+    if (!w_logical || !w_packed || K <= 0 || N <= 0 || (K & 1) || (N % 8)) return W4A16_ERR_INVALID_ARG;
+    if (!aligned16(w_packed)) return W4A16_ERR_INVALID_ARG;
+    const int kchunks = cdiv(K, kKC), n_tiles = cdiv(N, kBN);
+    const long long total = static_cast<long long>(n_tiles) * kchunks * 2048;
+    const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 65535LL * 8));
+    repack_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        w_logical, K, N, kchunks, n_tiles, static_cast<uint32_t*>(w_packed));
+    return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+}
+
+w4a16_status w4a16_msd_matmul(const void* x, const void* w_packed, const void* scale, int M, int K, int N,
+                              int group_size, void* y, void* workspace, size_t workspace_bytes,
+                              w4a16_stream_t stream)
+{
+    return dense_matmul(W4A16_OP_MSD, x, w_packed, scale, M, K, N, group_size, y, workspace, workspace_bytes,
+                        reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr, 0, 0, 0, 0);
+}
+
+w4a16_status w4a16_dequant_matmul(const void* x, const void* w_packed, const void* scale, int M, int K, int N,
+                                  int group_size, void* y, void* workspace, size_t workspace_bytes,
+                                  w4a16_stream_t stream)
+{
+    return dense_matmul(W4A16_OP_DEQUANT, x, w_packed, scale, M, K, N, group_size, y, workspace,
+                        workspace_bytes, reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr, 0, 0, 0, 0);
+}
+
+w4a16_status w4a16_msd_debug_yint(const void* x, const void* w_packed, int M, int K, int N, int group_size,
+                                  int m0, int m1, int n0, int n1, int32_t* yint, float* amax, void* workspace,
+                                  size_t workspace_bytes, w4a16_stream_t stream)
+{
+    if (!yint || !amax) return W4A16_ERR_INVALID_ARG;
+    if (m0 < 0 || m1 <= m0 || m1 > M || n0 < 0 || n1 <= n0 || n1 > N) return W4A16_ERR_INVALID_ARG;
+    // equation 9 needs no scale
+    return dense_matmul(W4A16_OP_MSD, x, w_packed, nullptr, M, K, N, group_size, nullptr, workspace,
+                        workspace_bytes, reinterpret_cast<cudaStream_t>(stream), yint, amax, m0, m1, n0, n1);
+}
+
+w4a16_status w4a16_grouped_matmul(int op, const void* x, const void* const* w_packed, const void* const* scale,
+                                  const int32_t* offsets, int E, int T, int K, int N, int group_size, void* y,
+                                  void* workspace, size_t workspace_bytes, w4a16_stream_t stream)
+{
+    if (op != W4A16_OP_MSD && op != W4A16_OP_DEQUANT) return W4A16_ERR_INVALID_ARG;
+    if (E < 1 || E > kMaxExperts) return W4A16_ERR_INVALID_ARG;
+    w4a16_status st = check_shape(T, K, N, group_size);
+    if (st != W4A16_OK) return st;
+    if (op == W4A16_OP_MSD && group_size > kMaxGroupMsd) return W4A16_ERR_UNSUPPORTED;
+    if (T == 0) return W4A16_OK;
+    if (!x || !w_packed || !scale || !offsets || !y || !workspace) return W4A16_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(workspace)) return W4A16_ERR_INVALID_ARG;
+    for (int e = 0; e < E; ++e)
+        if (!w_packed[e] || !scale[e] || !aligned16(w_packed[e]) || !aligned16(scale[e]))
+            return W4A16_ERR_INVALID_ARG;
+    const Shape s = grouped_shape(op, T, K, N, group_size, E);
+    const WsLayout L = ws_layout(op, s, T, K, N, group_size);
+    if (workspace_bytes < L.total) return W4A16_ERR_WORKSPACE;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+
+    GemmParams P;
+    base_params(P, T, K, N, group_size, s, workspace);
+    uint8_t* wsb = static_cast<uint8_t*>(workspace);
+    P.E = E;
+    P.offsets = offsets;
+    for (int e = 0; e < E; ++e) {
+        P.w[e] = static_cast<const uint8_t*>(w_packed[e]);
+        P.scale[e] = static_cast<const __half*>(scale[e]);
+    }
+    P.y = static_cast<__half*>(y);
+    CUtensorMap map;
+    if (op == W4A16_OP_MSD) {
+        int8_t* xq = reinterpret_cast<int8_t*>(wsb + L.xq);
+        float* amax = reinterpret_cast<float*>(wsb + L.amax);
+        st = launch_expand(x, T, K, group_size, xq, amax, cs);
+        if (st != W4A16_OK) return st;
+        P.amax = amax;
+        if (!make_map(&map, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, 3 * T, kKC, s.TT)) return W4A16_ERR_CUDA;
+    } else {
+        if (!make_map(&map, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K, T, 64, s.TT)) return W4A16_ERR_CUDA;
+    }
+    dim3 grid(s.n_tiles, 1, s.t_slots);
+    return launch_for(op, s.TT, map, P, grid, cs);
+}
+
+w4a16_status w4a16_read_status(const void* workspace, w4a16_stream_t stream, uint32_t* status)
+{
+    if (!workspace || !status) return W4A16_ERR_INVALID_ARG;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(status, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+        return W4A16_ERR_CUDA;
+    if (cudaStreamSynchronize(cs) != cudaSuccess) return W4A16_ERR_CUDA;
+    return (*status & W4A16_DEVICE_TIMEOUT) ? W4A16_ERR_TIMEOUT : W4A16_OK;
+}
+
+void w4a16_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns); }
+
+w4a16_status w4a16_selftest_wait_timeout(void* workspace, uint64_t timeout_ns, w4a16_stream_t stream)
+{
+    if (!workspace || !aligned16(workspace)) return W4A16_ERR_INVALID_ARG;
+    selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(static_cast<uint32_t*>(workspace),
+                                                                             timeout_ns);
+    return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+}
+
+}  // extern "C"
