@@ -24,7 +24,8 @@
  * Conventions for every entry point
  *  - Pointers marked "device" are CUDA device pointers owned by the caller;
  *    pointers marked "host" are host memory owned by the caller.  The
- *    library allocates no memory and keeps no state between calls.
+ *    library allocates no memory and keeps no state between calls (the one
+ *    exception, w4a16_msd_matmul_noalloc, describes its own array).
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *    stream).  No entry point synchronises the stream, except
  *    w4a16_read_status, which says so.
@@ -159,6 +160,34 @@ w4a16_status w4a16_msd_debug_yint(const void* x, const void* w_packed, int M, in
                                   int N, int group_size, int m0, int m1, int n0, int n1,
                                   int32_t* yint, float* amax, void* workspace,
                                   size_t workspace_bytes, w4a16_stream_t stream);
+
+/* MSD matmul for callers that cannot allocate device memory.
+ * No counterpart in the paper: this entry point exists for callers that have
+ * no way to obtain scratch memory -- for instance a plug-in running inside a
+ * host program whose memory pool owns the whole device, or a latency-critical
+ * path where cudaMalloc's implicit device synchronisation is not acceptable.
+ * It computes exactly what w4a16_msd_matmul computes (same kernels, same
+ * arguments minus the workspace) but keeps its scratch (the expanded
+ * activations, A_max, split-K partial sums and counters, status word) in one
+ * array of W4A16_NOALLOC_SCRATCH_BYTES bytes that the library declares in
+ * device memory; every GPU that loads the library holds that array until the
+ * process exits.  It allocates nothing and calls no allocating routine.
+ *  - Calls whose scratch would exceed the array (see w4a16_workspace_size
+ *    with W4A16_OP_MSD and E = 1) return W4A16_ERR_WORKSPACE and launch nothing.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - All calls share the one array and it keeps the previous call's
+ *    contents; each call zeroes the parts that must start at zero (status
+ *    word, split-K counters) on `stream` before its kernels run.  Calls that
+ *    may overlap on the GPU (different streams, or different host threads)
+ *    race on the array: serialise them.
+ *  - A device-side wait timeout is recorded only in the array's status word,
+ *    which this entry point does not report. */
+#define W4A16_NOALLOC_SCRATCH_BYTES (8u << 20)
+w4a16_status w4a16_msd_matmul_noalloc(const void* x, const void* w_packed, const void* scale,
+                                      int M, int K, int N, int group_size, void* y,
+                                      w4a16_stream_t stream);
 
 /* Copy the device status word at the start of `workspace` into *status
  * (0 = no device error; W4A16_DEVICE_TIMEOUT bit = a bounded wait expired).

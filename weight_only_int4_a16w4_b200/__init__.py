@@ -55,6 +55,8 @@ _lib.w4a16_grouped_matmul.restype = _I
 _lib.w4a16_grouped_matmul.argtypes = [_I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]
 _lib.w4a16_msd_debug_yint.restype = _I
 _lib.w4a16_msd_debug_yint.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]
+_lib.w4a16_msd_matmul_noalloc.restype = _I
+_lib.w4a16_msd_matmul_noalloc.argtypes = [_P, _P, _P, _I, _I, _I, _I, _P, _P]
 _lib.w4a16_read_status.restype = _I
 _lib.w4a16_read_status.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_uint32)]
 _lib.w4a16_set_wait_timeout_ns.restype = None
@@ -136,6 +138,16 @@ def w4a16_msd_debug_yint(x, w_packed, M, K, N, group_size, m0, m1, n0, n1, yint,
     _check(_lib.w4a16_msd_debug_yint(_ptr(x), _ptr(w_packed), M, K, N, group_size, m0, m1, n0, n1, _ptr(yint),
                                      _ptr(amax), _ptr(workspace), wb, _stream(stream)),
            "w4a16_msd_debug_yint")
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def w4a16_msd_matmul_noalloc(x, w_packed, scale, M, K, N, group_size, y, stream=None):
+    """MSD matmul whose scratch lives in the library's own device array (no
+    workspace argument; for callers that cannot allocate device memory)."""
+    _check(_lib.w4a16_msd_matmul_noalloc(_ptr(x), _ptr(w_packed), _ptr(scale), M, K, N, group_size, _ptr(y),
+                                         _stream(stream)), "w4a16_msd_matmul_noalloc")
 
 
 def w4a16_read_status(workspace, stream=None) -> int:

@@ -298,6 +298,32 @@ w4a16_status dense_matmul(int op, const void* x, const void* w_packed, const voi
 
 }  // namespace
 
+// Scratch of w4a16_msd_matmul_noalloc: one array in device memory per GPU
+// that loads the library.  Host code must not use the symbol itself as an
+// address; the device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[W4A16_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device with that device current.  nullptr on failure.
+void* noalloc_scratch()
+{
+    static std::mutex mu;
+    static void* addr[64] = {nullptr};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return nullptr;
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
+}  // namespace
+
 // =================================================================== C ABI
 
 extern "C" {
@@ -416,6 +442,25 @@ w4a16_status w4a16_grouped_matmul(int op, const void* x, const void* const* w_pa
     }
     dim3 grid(s.n_tiles, 1, s.t_slots);
     return launch_for(op, s.TT, map, P, grid, cs);
+}
+
+w4a16_status w4a16_msd_matmul_noalloc(const void* x, const void* w_packed, const void* scale, int M, int K, int N,
+                                      int group_size, void* y, w4a16_stream_t stream)
+{
+    size_t need = 0;
+    w4a16_status st = w4a16_workspace_size(W4A16_OP_MSD, M, K, N, group_size, 1, &need);
+    if (st != W4A16_OK) return st;
+    if (need > W4A16_NOALLOC_SCRATCH_BYTES) return W4A16_ERR_WORKSPACE;
+    if (M == 0) return W4A16_OK;
+    void* ws = noalloc_scratch();
+    if (ws == nullptr) return W4A16_ERR_CUDA;
+    // the status word and the split-K arrival counters must start at zero
+    const Shape s = dense_shape(W4A16_OP_MSD, M, K, N, group_size);
+    const WsLayout L = ws_layout(W4A16_OP_MSD, s, M, K, N, group_size);
+    const size_t zero_bytes = (s.splits > 1) ? L.partial : kHeaderBytes;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws, 0, zero_bytes, cs) != cudaSuccess) return W4A16_ERR_CUDA;
+    return w4a16_msd_matmul(x, w_packed, scale, M, K, N, group_size, y, ws, W4A16_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 w4a16_status w4a16_read_status(const void* workspace, w4a16_stream_t stream, uint32_t* status)
