@@ -13,7 +13,7 @@ import ctypes
 import os
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libw4a16.so")
+LIB_PATH = os.environ.get("W4A16_LIBRARY") or os.path.join(_PKG, "libw4a16.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(

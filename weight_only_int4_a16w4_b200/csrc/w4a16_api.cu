@@ -8,6 +8,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -15,6 +16,19 @@
 #include "w4a16_kernels.cuh"
 
 using namespace w4a16;
+
+#ifdef W4A16_TRACE
+extern "C" int w4a16_trace_copy(unsigned long long* host, int n)
+{
+    if (n > 1024 * 64) n = 1024 * 64;
+    return cudaMemcpyFromSymbol(host, w4a16_trace_buf, sizeof(unsigned long long) * n) == cudaSuccess ? 0 : 1;
+}
+extern "C" int w4a16_trace_clear(const unsigned long long* zeros, int n)
+{
+    if (n > 1024 * 64) n = 1024 * 64;
+    return cudaMemcpyToSymbol(w4a16_trace_buf, zeros, sizeof(unsigned long long) * n) == cudaSuccess ? 0 : 1;
+}
+#endif
 
 namespace {
 
@@ -80,9 +94,6 @@ bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int el
 
 // ---------------------------------------------------------------- launch shapes
 
-// Kernel instances:  (variant, token tile, load stages, A stages, CTAs/SM)
-//   decode (M <= 16):  MSD <kMsd,16,7,4,2>   DEQUANT <kDeq,16,8,2,2>
-//   larger M:          MSD <kMsd,64,4,4,1>   DEQUANT <kDeq,128,2,2,2>
 struct Shape {
     int TT;
     int splits;
@@ -100,24 +111,18 @@ int tile_tokens(int op, int M)
     return op == W4A16_OP_MSD ? 64 : 128;
 }
 
-// Split-K factor for a dense call: spread (column tiles x token tiles) work
-// over every SM when there are fewer tiles than SMs, minimising the number
-// of chunk-steps on the busiest SM (2 resident CTAs per SM for the decode tile).
-int choose_splits(int tiles, int units, int resident)
+// Split-K factor for a decode-sized dense call: the CTAs of one column tile
+// split K among themselves and reduce through distributed shared memory
+// (a cluster of `splits` CTAs).  At most one CTA per SM, so that the next
+// kernel in the stream can already occupy the second slot (programmatic
+// dependent launch); the largest factor that keeps all CTAs in one wave.
+int choose_splits(int tiles, int units)
 {
-    const int slots = std::max(1, sm_count() * resident);
-    if (tiles >= sm_count() || units <= 1) return 1;
-    long best_cost = -1;
+    const int sms = sm_count();
+    if (tiles >= sms || units <= 1) return 1;
     int best = 1;
-    for (int s = 1; s <= units; ++s) {
-        const long ctas = static_cast<long>(tiles) * s;
-        const long waves = (ctas + slots - 1) / slots;
-        const long cost = waves * ((units + s - 1) / s);
-        if (best_cost < 0 || cost < best_cost) {
-            best_cost = cost;
-            best = s;
-        }
-    }
+    for (int s = 2; s <= std::min(units, 8); ++s)
+        if (static_cast<long>(tiles) * s <= sms) best = s;
     return best;
 }
 
@@ -130,7 +135,7 @@ Shape dense_shape(int op, int M, int K, int N, int g)
     s.t_slots = std::max(1, cdiv(M, s.TT));
     s.unit = std::max(1, g / kKC);
     const int units = cdiv(s.kchunks, s.unit);
-    s.splits = small_tile(op, M) ? choose_splits(s.n_tiles * s.t_slots, units, 2) : 1;
+    s.splits = small_tile(op, M) ? choose_splits(s.n_tiles * s.t_slots, units) : 1;
     return s;
 }
 
@@ -147,19 +152,15 @@ Shape grouped_shape(int op, int T, int K, int N, int g, int E)
 }
 
 struct WsLayout {
-    size_t counters = 0, partial = 0, xq = 0, amax = 0, total = 0;
+    size_t xq = 0, amax = 0, total = 0;
 };
 
 WsLayout ws_layout(int op, const Shape& s, int M, int K, int N, int g)
 {
+    (void)s;
+    (void)N;
     WsLayout L;
     size_t off = kHeaderBytes;
-    if (s.splits > 1) {
-        L.counters = off;
-        off += align256(static_cast<size_t>(s.t_slots) * s.n_tiles * 4);
-        L.partial = off;
-        off += align256(static_cast<size_t>(s.splits) * M * N * 4);
-    }
     if (op == W4A16_OP_MSD) {
         L.xq = off;
         off += align256(static_cast<size_t>(3) * M * K);
@@ -182,29 +183,99 @@ w4a16_status check_shape(int M, int K, int N, int g)
 
 // ---------------------------------------------------------------- kernel launch
 
-template <int VAR, int TT, int LS, int AS, int MINB>
+bool use_pdl()
+{
+    static int v = -1;
+    if (v < 0) {
+        const char* e = std::getenv("W4A16_PDL");
+        v = (e && e[0] == '0') ? 0 : 1;
+    }
+    return v == 1;
+}
+
+template <int VAR, int TT, int ST, int WST, int NCONV, int NEPI, int NISS, bool SEPI, bool DBG = false>
 w4a16_status launch_gemm(const CUtensorMap& map, const GemmParams& P, dim3 grid, cudaStream_t stream)
 {
-    using C = GemmCfg<VAR, TT, LS, AS>;
-    auto kern = gemm_kernel<VAR, TT, LS, AS, MINB>;
+    using C = GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, SEPI>;
+    auto kern = gemm_kernel<VAR, TT, ST, WST, NCONV, NEPI, NISS, SEPI, DBG>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
         attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     });
     if (attr_err != cudaSuccess) return W4A16_ERR_CUDA;
-    kern<<<grid, kThreads, C::kSmem, stream>>>(map, P);
-    return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+    // split-K reduces through the decode tile's own partial buffer
+    if (P.splits > 1 && (C::kRedBytes == 0 || P.splits > 16)) return W4A16_ERR_UNSUPPORTED;
+    if (P.issuers < 1 || P.issuers > NISS || ST % P.issuers != 0) return W4A16_ERR_UNSUPPORTED;
+    if (C::kGroupAcc && P.issuers > 1 && P.g != kKC) return W4A16_ERR_UNSUPPORTED;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(C::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attrs[2];
+    int na = 0;
+    if (use_pdl()) {
+        attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attrs[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    if (P.splits > 1) {   // the split-K CTAs of one tile form a cluster (see gemm_kernel)
+        attrs[na].id = cudaLaunchAttributeClusterDimension;
+        attrs[na].val.clusterDim.x = 1;
+        attrs[na].val.clusterDim.y = static_cast<unsigned>(P.splits);
+        attrs[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    cfg.attrs = attrs;
+    cfg.numAttrs = na;
+    if (cudaLaunchKernelEx(&cfg, kern, map, P) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return W4A16_ERR_CUDA;
+    }
+    return W4A16_OK;
 }
 
+// Kernel instances (variant, token tile, operand stages, weight stages,
+// converter groups, epilogue groups, MMA issuers, scale in the epilogue);
+// one CTA per SM, 512 Tensor Memory columns.
+//   decode (M <= 16): MSD <16, 8, 12, 2, 1, 4>   DEQUANT <16, 4, 12, 2, 1, 4, scale in epilogue>
+//     two converter groups and four MMA issuers: each small MMA (N = 48 / 16)
+//     holds its issuing thread for far longer than the tensor core needs, so
+//     the issue is spread over several warps
+//   larger M:         MSD <64, 4, 4, 1, 2, 1>   DEQUANT <128, 4, 4, 1, 1, 1>
+//     MSD's per-group combine is the bottleneck: two epilogue groups
 w4a16_status launch_for(int op, int TT, const CUtensorMap& map, const GemmParams& P, dim3 grid, cudaStream_t s)
 {
     if (op == W4A16_OP_MSD) {
-        if (TT == 16) return launch_gemm<kMsd, 16, 7, 4, 2>(map, P, grid, s);
-        return launch_gemm<kMsd, 64, 4, 4, 1>(map, P, grid, s);
+        // the Y_int debug window is a separate instance, off the hot kernels
+        if (P.dbg_yint != nullptr) {
+            if (TT == 16) return launch_gemm<kMsd, 16, 8, 12, 2, 1, 4, false, true>(map, P, grid, s);
+            return launch_gemm<kMsd, 64, 4, 4, 1, 2, 1, false, true>(map, P, grid, s);
+        }
+        if (TT == 16) return launch_gemm<kMsd, 16, 8, 12, 2, 1, 4, false>(map, P, grid, s);
+        return launch_gemm<kMsd, 64, 4, 4, 1, 2, 1, false>(map, P, grid, s);
     }
-    if (TT == 16) return launch_gemm<kDeq, 16, 8, 2, 2>(map, P, grid, s);
-    return launch_gemm<kDeq, 128, 2, 2, 2>(map, P, grid, s);
+    if (TT == 16) return launch_gemm<kDeq, 16, 4, 12, 2, 1, 4, true>(map, P, grid, s);
+    return launch_gemm<kDeq, 128, 4, 4, 1, 1, 1, false>(map, P, grid, s);
+}
+
+template <int VPL>
+cudaError_t launch_expand_vpl(int blocks, const __half* x, int M, int K, int g, int8_t* xq, float* amax,
+                              cudaStream_t s)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(blocks, 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = use_pdl() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, expand_kernel<VPL>, x, M, K, g, xq, amax);
 }
 
 w4a16_status launch_expand(const void* x, int M, int K, int g, int8_t* xq, float* amax, cudaStream_t s)
@@ -212,15 +283,20 @@ w4a16_status launch_expand(const void* x, int M, int K, int g, int8_t* xq, float
     const long long warps = static_cast<long long>(M) * (K / g);
     const int blocks = static_cast<int>((warps + 7) / 8);
     const __half* xh = static_cast<const __half*>(x);
+    cudaError_t e;
     switch (g / 32) {
-        case 1: expand_kernel<1><<<blocks, 256, 0, s>>>(xh, M, K, g, xq, amax); break;
-        case 2: expand_kernel<2><<<blocks, 256, 0, s>>>(xh, M, K, g, xq, amax); break;
-        case 4: expand_kernel<4><<<blocks, 256, 0, s>>>(xh, M, K, g, xq, amax); break;
-        case 8: expand_kernel<8><<<blocks, 256, 0, s>>>(xh, M, K, g, xq, amax); break;
-        case 16: expand_kernel<16><<<blocks, 256, 0, s>>>(xh, M, K, g, xq, amax); break;
+        case 1: e = launch_expand_vpl<1>(blocks, xh, M, K, g, xq, amax, s); break;
+        case 2: e = launch_expand_vpl<2>(blocks, xh, M, K, g, xq, amax, s); break;
+        case 4: e = launch_expand_vpl<4>(blocks, xh, M, K, g, xq, amax, s); break;
+        case 8: e = launch_expand_vpl<8>(blocks, xh, M, K, g, xq, amax, s); break;
+        case 16: e = launch_expand_vpl<16>(blocks, xh, M, K, g, xq, amax, s); break;
         default: return W4A16_ERR_UNSUPPORTED;
     }
-    return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return W4A16_ERR_CUDA;
+    }
+    return W4A16_OK;
 }
 
 void base_params(GemmParams& P, int M, int K, int N, int g, const Shape& s, void* ws)
@@ -237,6 +313,7 @@ void base_params(GemmParams& P, int M, int K, int N, int g, const Shape& s, void
     P.splits = s.splits;
     P.unit = s.unit;
     P.E = 1;
+    P.issuers = 1;
     P.status = static_cast<uint32_t*>(ws);
     P.timeout_ns = g_timeout_ns.load();
     P.write_y = 1;
@@ -268,10 +345,6 @@ w4a16_status dense_matmul(int op, const void* x, const void* w_packed, const voi
     P.w[0] = static_cast<const uint8_t*>(w_packed);
     P.scale[0] = static_cast<const __half*>(scale);
     P.y = static_cast<__half*>(y);
-    if (s.splits > 1) {
-        P.counters = reinterpret_cast<uint32_t*>(wsb + L.counters);
-        P.partial = reinterpret_cast<float*>(wsb + L.partial);
-    }
     if (debug) {
         P.write_y = 0;
         P.dbg_yint = dbg_yint;
@@ -292,6 +365,10 @@ w4a16_status dense_matmul(int op, const void* x, const void* w_packed, const voi
     } else {
         if (!make_map(&map, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K, M, 64, s.TT)) return W4A16_ERR_CUDA;
     }
+    // four MMA issuers on the decode tile when a group is exactly one
+    // 128-deep chunk: each issuer then owns one of the per-group
+    // accumulator buffers
+    if (s.TT == 16) P.issuers = (g == kKC) ? 4 : 1;
     dim3 grid(s.n_tiles, s.splits, s.t_slots);
     return launch_for(op, s.TT, map, P, grid, stream);
 }
@@ -454,12 +531,9 @@ w4a16_status w4a16_msd_matmul_noalloc(const void* x, const void* w_packed, const
     if (M == 0) return W4A16_OK;
     void* ws = noalloc_scratch();
     if (ws == nullptr) return W4A16_ERR_CUDA;
-    // the status word and the split-K arrival counters must start at zero
-    const Shape s = dense_shape(W4A16_OP_MSD, M, K, N, group_size);
-    const WsLayout L = ws_layout(W4A16_OP_MSD, s, M, K, N, group_size);
-    const size_t zero_bytes = (s.splits > 1) ? L.partial : kHeaderBytes;
+    // the status word must start at zero
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-    if (cudaMemsetAsync(ws, 0, zero_bytes, cs) != cudaSuccess) return W4A16_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, kHeaderBytes, cs) != cudaSuccess) return W4A16_ERR_CUDA;
     return w4a16_msd_matmul(x, w_packed, scale, M, K, N, group_size, y, ws, W4A16_NOALLOC_SCRATCH_BYTES, stream);
 }
 

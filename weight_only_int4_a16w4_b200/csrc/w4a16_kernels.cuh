@@ -35,11 +35,31 @@
 //               double-buffered accumulators); fp16 store or split-K partial.
 #pragma once
 
+#ifndef W4A16_ROLE_UNROLL
+#define W4A16_ROLE_UNROLL _Pragma("unroll")
+#endif
+
 #include <cuda_fp16.h>
 
 #include <cstdint>
 
 #include "sm100_ptx.cuh"
+
+// Optional timeline tracing (build with -DW4A16_TRACE): selected threads
+// stamp SM clock cycles at pipeline events into a per-CTA row of
+// w4a16_trace_buf, read back by the trace build's w4a16_trace_copy.
+#ifdef W4A16_TRACE
+__device__ unsigned long long w4a16_trace_buf[1024 * 64];
+#define W4A16_TRACE_AT(slot)                                                                                  \
+    do {                                                                                                      \
+        const unsigned cta_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);                \
+        if (cta_ < 1024 && (slot) < 64) w4a16_trace_buf[cta_ * 64 + (slot)] = clock64();                    \
+    } while (0)
+#else
+#define W4A16_TRACE_AT(slot) \
+    do {                     \
+    } while (0)
+#endif
 
 namespace w4a16 {
 
@@ -47,7 +67,6 @@ constexpr int kBN = 128;                 // output columns per tile (MMA M)
 constexpr int kKC = 128;                 // K per pipeline stage
 constexpr int kWStage = kBN * kKC / 2;   // packed bytes per (tile, chunk): 8192
 constexpr int kMaxExperts = 64;
-constexpr int kThreads = 320;
 constexpr int kMaxGroupMsd = 512;        // expand_kernel: at most 16 values per lane
 
 enum Variant { kMsd = 0, kDeq = 1 };
@@ -66,13 +85,12 @@ struct GemmParams {
     int t_slots;    // grid.z: token tiles (dense) or tile slots (grouped)
     int splits;     // split-K factor (dense); 1 = no split
     int unit;       // chunks per split unit (keeps splits on group boundaries)
+    int issuers;    // MMA issuer warps in use (1 or 2)
     int E;
     const int32_t* offsets;                 // grouped: device [E+1]; dense: nullptr
     const uint8_t* w[kMaxExperts];          // packed weights per expert
     const __half* scale[kMaxExperts];       // [G][N] per expert
     __half* y;                              // [M][N]
-    float* partial;                         // split-K: [splits][M][N]
-    uint32_t* counters;                     // split-K: [t_slots][n_tiles]
     const float* amax;                      // MSD: [G][M]
     uint32_t* status;
     unsigned long long timeout_ns;
@@ -82,25 +100,64 @@ struct GemmParams {
     int dbg_m0, dbg_m1, dbg_n0, dbg_n1;
 };
 
-template <int VAR, int TT, int LS, int AS>
+// Compile-time shape of one gemm_kernel instance.
+//   TT     tokens per tile (MMA N for DEQUANT, N / 3 for MSD)
+//   ST     operand stages: stage s holds the activation tile of a chunk in
+//          shared memory and its converted A operand in Tensor Memory
+//   WST    weight stages (shared memory only): the packed weight chunk and
+//          (optionally) its scale rows; deeper than ST so that enough weight
+//          bytes are in flight while Tensor Memory bounds ST
+//   NCONV  converter warp groups (4 warps each) taking alternate chunks
+//   NEPI   epilogue warp groups (4 warps each) splitting the tile's tokens
+//   NISS   MMA issuer warps available (the launch may use fewer)
+//   SEPI   DEQUANT only: apply the group scale in the epilogue, to per-group
+//          fp32 accumulators (decode tiles), instead of in the converter
+//          (W' = fp16(scale * w), one accumulator over all of K)
+//   DBG    write the MSD Y_int debug window
+// Warps: 0 weight producer; 1 activation producer; 2 .. 1+NISS MMA issuers;
+// the control block is padded to a multiple of 4 warps; then the converter
+// groups, then the epilogue groups.  Chunk i lives in stage i % ST and is
+// served by converter group i % NCONV and issuer i % issuers; ST is a
+// multiple of both, so every stage is always served by the same group and no
+// waiter can run two phases ahead of a barrier.  Group-accumulator mode keeps
+// NBUF = max(2, NISS) accumulator buffers, buffer = group % NBUF; with several
+// issuers a group is one chunk, so each issuer owns one buffer.
+template <int VAR, int TT, int ST, int WST, int NCONV, int NEPI, int NISS, bool SEPI>
 struct GemmCfg {
     static constexpr bool kIsMsd = VAR == kMsd;
-    static constexpr int kMmaN = kIsMsd ? 3 * TT : TT;
+    static constexpr bool kGroupAcc = kIsMsd || SEPI;      // per-group accumulators + per-group epilogue
+    static constexpr int kVals = kIsMsd ? 3 : 1;           // accumulators per token (Y1..Y3 or y)
+    static constexpr int kMmaN = kVals * TT;
     static constexpr int kBBytes = kIsMsd ? 3 * TT * 128 : 2 * TT * 128;   // activation tile per stage
-    static constexpr int kSBytes = kIsMsd ? 0 : 1024;                      // up to 4 scale rows
-    static constexpr int kStage = kBBytes + kWStage + kSBytes;
+    static constexpr int kSBytes = (kIsMsd || SEPI) ? 0 : 1024;            // up to 4 scale rows
+    static constexpr int kStage = kBBytes;                                 // operand stage (shared part)
+    static constexpr int kWSlot = kWStage + kSBytes;                       // weight stage
+    static constexpr int kMaxIssuers = NISS;
+    static constexpr int kNBuf = kGroupAcc ? (NISS > 2 ? NISS : 2) : 1;
     static constexpr int kAccStride = ((kMmaN + 31) / 32) * 32;
-    static constexpr int kNAcc = kIsMsd ? 2 : 1;
+    static constexpr int kAccCols = kNBuf * kAccStride;
     static constexpr int kACols = kIsMsd ? 32 : 64;                        // A operand per stage
-    static constexpr int kColsUsed = kNAcc * kAccStride + AS * kACols;
+    static constexpr int kColsUsed = kAccCols + ST * kACols;
     static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
                                    : kColsUsed <= 256 ? 256 : 512;
-    static constexpr int kNumBars = 2 * LS + 2 * AS + 2 * kNAcc + 1;
-    static constexpr int kSmem = LS * kStage + 1024 + 8 * kNumBars + 64;
+    static constexpr int kCtrlWarps = ((2 + NISS + 3) / 4) * 4;
+    static constexpr int kConvWarp0 = kCtrlWarps;
+    static constexpr int kEpiWarp0 = kCtrlWarps + 4 * NCONV;
+    static constexpr int kWarps = kCtrlWarps + 4 * NCONV + 4 * NEPI;
+    static constexpr int kThreads = 32 * kWarps;
+    static constexpr int kEpiThreads = 128 * NEPI;
+    static constexpr int kTokPerEpi = TT / NEPI;
+    static constexpr int kRedBytes = TT == 16 ? TT * kBN * 4 + 256 : 0;     // split-K partials (decode tile only)
+    static constexpr int kNumBars = 3 * ST + 2 * WST + 2 * kNBuf + kMaxIssuers;
+    static constexpr int kSmem = ST * kStage + WST * kWSlot + kRedBytes + 1024 + 8 * kNumBars + 16 + 2 * TT * 4 + 16;
     static_assert(kColsUsed <= 512, "Tensor Memory overflow");
     static_assert(kMmaN % 16 == 0 && kMmaN >= 16 && kMmaN <= 256, "MMA N out of range");
-    static_assert(TT % 16 == 0, "token tile must be a multiple of 16");
-    static_assert(kStage % 1024 == 0, "stages must keep 1024-byte alignment");
+    static_assert(TT % 16 == 0 && kTokPerEpi % 16 == 0, "token tile must split into 16-token pieces");
+    static_assert(kStage % 1024 == 0 && kWSlot % 1024 == 0, "stages must keep 1024-byte alignment");
+    static_assert(kSmem <= 227 * 1024, "shared memory overflow");
+    static_assert(ST % NCONV == 0 && ST % NISS == 0 && WST % NCONV == 0, "stages must split evenly over the groups");
+    static_assert(NISS == 1 || NISS == 2 || NISS == 4, "1, 2 or 4 MMA issuers");
+    static_assert(!SEPI || !kIsMsd, "SEPI is a DEQUANT option");
 };
 
 // ------------------------------------------------------------------ helpers
@@ -110,18 +167,40 @@ __device__ __forceinline__ uint32_t pack_half2_bits(__half2 h)
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Eight int4 weights of one packed word -> four fp16 pairs scaled by s.
-// Word layout (written by repack_kernel): nibble 4*i..4*i+3 (i < 4) holds
-// element 2i, nibble 16+4*i.. holds element 2i+1, each as (w + 8).  Pair i
-// is built from the binary16 format: 0x6400 | u is the half 1024 + u.
-__device__ __forceinline__ void dequant_word(uint32_t q, __half2 s2, uint32_t* out4)
+// Eight int4 weights of one packed word -> four fp16 pairs (w exactly).
+// Word layout (written by repack_kernel): bits 4i..4i+3 (i < 4) hold element
+// 2i, bits 16+4i.. hold element 2i+1, each as u = w + 8.  From the binary16
+// format: 0x6400 | u is the half 1024 + u, and 0x6400 | (u << 4) is
+// 1024 + 16u.  So pair 0 is (0x6400|u) - 1032 and pair 1 is
+// (0x6400|16u) * (1/16) - 72, both exact (one rounding of an exact value);
+// pairs 2 and 3 repeat this on the word shifted by 8.  9 instructions.
+__device__ __forceinline__ void int4_to_half2x4(uint32_t q, uint32_t* out4)
 {
-    const __half2 bias = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));  // 1032
+    const __half2 k1032 = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));   // 1032
+    const __half2 k16th = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));   // 1/16
+    const __half2 km72 = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));    // -72
+    const uint32_t q8 = q >> 8;
+    uint32_t h0 = (q & 0x000F000Fu) | 0x64006400u;
+    uint32_t h1 = (q & 0x00F000F0u) | 0x64006400u;
+    uint32_t h2 = (q8 & 0x000F000Fu) | 0x64006400u;
+    uint32_t h3 = (q8 & 0x00F000F0u) | 0x64006400u;
+    const __half2 w0 = __hsub2(*reinterpret_cast<__half2*>(&h0), k1032);
+    const __half2 w1 = __hfma2(*reinterpret_cast<__half2*>(&h1), k16th, km72);
+    const __half2 w2 = __hsub2(*reinterpret_cast<__half2*>(&h2), k1032);
+    const __half2 w3 = __hfma2(*reinterpret_cast<__half2*>(&h3), k16th, km72);
+    out4[0] = pack_half2_bits(w0);
+    out4[1] = pack_half2_bits(w1);
+    out4[2] = pack_half2_bits(w2);
+    out4[3] = pack_half2_bits(w3);
+}
+
+// The same, each pair multiplied by the group scale: fp16(scale * w).
+__device__ __forceinline__ void int4_to_half2x4_scaled(uint32_t q, __half2 s2, uint32_t* out4)
+{
+    int4_to_half2x4(q, out4);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        uint32_t h = ((q >> (4 * i)) & 0x000F000Fu) | 0x64006400u;
-        __half2 v = __hsub2(*reinterpret_cast<__half2*>(&h), bias);   // exact: w in [-8, 7]
-        v = __hmul2(v, s2);                                           // fp16(scale * w)
+        const __half2 v = __hmul2(*reinterpret_cast<__half2*>(&out4[i]), s2);
         out4[i] = pack_half2_bits(v);
     }
 }
@@ -193,6 +272,11 @@ __global__ void __launch_bounds__(256) expand_kernel(const __half* __restrict__ 
                                                      int8_t* __restrict__ xq, float* __restrict__ amax)
 {
     const int G = K / g;
+    // Let the matmul that consumes A_int launch now (it streams its weights
+    // meanwhile); x may come from the previous kernel, and the previous
+    // matmul may still read the A_int this kernel overwrites, so wait for it.
+    griddep_launch_dependents();
+    griddep_wait();
     const long long warp = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (warp >= static_cast<long long>(M) * G) return;
@@ -268,41 +352,47 @@ __device__ __forceinline__ bool resolve_tile(const GemmParams& P, int TT, TileCo
     return false;
 }
 
-// One output value for token row t0 + t, column n: fp16 y, or the fp32
-// split-K partial of this CTA's split.
-__device__ __forceinline__ void emit_value(const GemmParams& P, const TileCoord& tc, int n, int t, float v)
-{
-    if (P.splits == 1) {
-        if (P.write_y) P.y[static_cast<size_t>(tc.t0 + t) * P.N + n] = __float2half_rn(v);
-    } else {
-        P.partial[(static_cast<size_t>(tc.split) * P.M + tc.t0 + t) * P.N + n] = v;
-    }
-}
+// MSD accumulators start every group at this bias: an int32 accumulator
+// holding 0x4B400000 + Y reads, as a binary32, exactly 12582912 + Y for
+// |Y| < 2^22 (1.5 * 2^23 has a unit last place), so the epilogue turns Y into
+// a float with one exact subtraction instead of an int -> float conversion.
+constexpr uint32_t kAccBiasBits = 0x4B400000u;
+constexpr float kAccBias = 12582912.0f;
+// Equation 10 with 1/7.49 factored out: Y1 + Y2/14.98 + Y3/14.98^2.
+constexpr float kR2 = static_cast<float>(1.0 / 14.98);
+constexpr float kR3 = static_cast<float>(1.0 / (14.98 * 14.98));
 
-template <int VAR, int TT, int LS, int AS, int MINB>
-__global__ void __launch_bounds__(kThreads, MINB)
+template <int VAR, int TT, int ST, int WST, int NCONV, int NEPI, int NISS, bool SEPI, bool DBG>
+__global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, SEPI>::kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ GemmParams P)
 {
-    using C = GemmCfg<VAR, TT, LS, AS>;
+    using C = GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, SEPI>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + LS * C::kStage);
-    uint64_t* full_bar = bars;
-    uint64_t* empty_bar = full_bar + LS;
-    uint64_t* afull_bar = empty_bar + LS;
-    uint64_t* aempty_bar = afull_bar + AS;
-    uint64_t* accfull_bar = aempty_bar + AS;
-    uint64_t* accempty_bar = accfull_bar + C::kNAcc;
-    uint64_t* done_bar = accempty_bar + C::kNAcc;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
+    uint8_t* wsm = smem + ST * C::kStage;                              // weight slots
+    float* red = reinterpret_cast<float*>(wsm + WST * C::kWSlot);      // split-K partials pushed by the cluster
+    uint64_t* bars = reinterpret_cast<uint64_t*>(wsm + WST * C::kWSlot + C::kRedBytes);
+    uint64_t* bfull_bar = bars;                 // [ST] activation tile landed
+    uint64_t* sfree_bar = bfull_bar + ST;       // [ST] operand stage free again (MMA done)
+    uint64_t* afull_bar = sfree_bar + ST;       // [ST] A operand written to Tensor Memory
+    uint64_t* wfull_bar = afull_bar + ST;       // [WST] weight slot landed
+    uint64_t* wempty_bar = wfull_bar + WST;     // [WST] weight slot read by its converter group
+    uint64_t* accfull_bar = wempty_bar + WST;        // [kNBuf] accumulator ready for the epilogue
+    uint64_t* accempty_bar = accfull_bar + C::kNBuf; // [kNBuf] group accumulator read (and reset) by the epilogue
+    uint64_t* done_bar = accempty_bar + C::kNBuf;    // [kMaxIssuers] all MMAs of an issuer completed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + C::kMaxIssuers);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    volatile int* last_flag = abort_flag + 1;
+    // [2][TT] floats read as float4: round up to a 16-byte boundary (the
+    // barriers before it end on an 8-byte boundary only)
+    float* amax_sm = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(tmem_slot + 4) + 15) & ~uintptr_t(15));
 
     TileCoord tc;
     if (!resolve_tile(P, TT, tc)) return;          // uniform across the CTA
+    if (threadIdx.x == 0) W4A16_TRACE_AT(1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const int issuers = P.issuers;
 
     // K-chunk range of this split (split units keep groups whole).
     const int units = (P.kchunks + P.unit - 1) / P.unit;
@@ -310,23 +400,24 @@ __global__ void __launch_bounds__(kThreads, MINB)
     const int kc1 = min(P.kchunks, ((tc.split + 1) * units / P.splits) * P.unit);
     const int nchunks = kc1 - kc0;
     const int n0 = tc.n_tile * kBN;
+    const int grp0 = (kc0 * kKC) / P.g;                 // first group of this split
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < LS; ++s) {
-            mbar_init(smem_addr(&full_bar[s]), 1);
-            mbar_init(smem_addr(&empty_bar[s]), 1 + 4);
-        }
-        for (int s = 0; s < AS; ++s) {
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(smem_addr(&bfull_bar[s]), 1);
+            mbar_init(smem_addr(&sfree_bar[s]), 1);
             mbar_init(smem_addr(&afull_bar[s]), 4);
-            mbar_init(smem_addr(&aempty_bar[s]), 1);
         }
-        for (int b = 0; b < C::kNAcc; ++b) {
+        for (int w = 0; w < WST; ++w) {
+            mbar_init(smem_addr(&wfull_bar[w]), 1);
+            mbar_init(smem_addr(&wempty_bar[w]), 4);
+        }
+        for (int b = 0; b < C::kNBuf; ++b) {
             mbar_init(smem_addr(&accfull_bar[b]), 1);
-            mbar_init(smem_addr(&accempty_bar[b]), 4);
+            mbar_init(smem_addr(&accempty_bar[b]), 4 * NEPI);
         }
-        mbar_init(smem_addr(done_bar), 1);
+        for (int q = 0; q < C::kMaxIssuers; ++q) mbar_init(smem_addr(&done_bar[q]), 1);
         *abort_flag = 0;
-        *last_flag = 0;
         fence_barrier_init();
         prefetch_tensor_map(&tmap);
     }
@@ -334,135 +425,197 @@ __global__ void __launch_bounds__(kThreads, MINB)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // The next kernel in the stream may start launching now; it waits
+    // (griddep_wait) before touching anything this one writes.
+    if (threadIdx.x == 0) griddep_launch_dependents();
+    if (threadIdx.x == 0) W4A16_TRACE_AT(2);
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tmem_a0 = tmem + C::kNAcc * C::kAccStride;   // A operand stages
+    const uint32_t tmem_a0 = tmem + C::kAccCols;               // A operand stages
     const uint64_t tmo = P.timeout_ns;
 
-    if (warp == 0) {
-        // ============================ producer ============================
-        if (lane == 0 && nchunks > 0) {
+    if (warp == 0 || warp == 1) {
+        // ============================ producers ============================
+        // Warp 0 streams the packed weights (and the scale rows when the
+        // converter applies them) into the weight ring: constant inputs,
+        // fetched without waiting for the previous kernel.  Warp 1 brings the
+        // activation tiles (x, or the expansion kernel's A_int) into the
+        // operand stages once that kernel has finished.  The whole warp runs
+        // the loop (converged); lane 0 issues.
+        const bool weights = warp == 0;
+        if (nchunks > 0) {
             const uint8_t* wsrc = P.w[tc.e] + (static_cast<size_t>(tc.n_tile) * P.kchunks + kc0) * kWStage;
             const __half* ssrc = P.scale[tc.e];
             const uint32_t srow_bytes = static_cast<uint32_t>(min(kBN, P.N - n0)) * 2u;
+            if (!weights) griddep_wait();
+            const int ring = weights ? WST : ST;
+            uint64_t* fullb = weights ? wfull_bar : bfull_bar;
+            uint64_t* freeb = weights ? wempty_bar : sfree_bar;
             int issued = 0;
             for (int i = 0; i < nchunks; ++i) {
-                const int s = i % LS;
-                const uint32_t ph = (i / LS) & 1;
-                if (!mbar_wait(smem_addr(&empty_bar[s]), ph ^ 1, tmo, P.status, abort_flag)) break;
-                uint8_t* st = smem + s * C::kStage;
-                const uint32_t fb = smem_addr(&full_bar[s]);
-                const int kc = kc0 + i;
-                uint32_t bytes = kWStage + C::kBBytes;
-                int srows = 0, sgrp0 = 0;
-                if (!C::kIsMsd) {
-                    sgrp0 = (kc * kKC) / P.g;
-                    srows = (P.g >= kKC) ? 1 : min(kKC / P.g, P.G - sgrp0);
-                    bytes += srows * srow_bytes;
-                }
-                mbar_arrive_expect_tx(fb, bytes);
-                bulk_g2s(smem_addr(st + C::kBBytes), wsrc + static_cast<size_t>(i) * kWStage, kWStage, fb);
-                if (C::kIsMsd) {
+                const int s = i % ring;
+                const uint32_t ph = (i / ring) & 1;
+                if (!mbar_wait(smem_addr(&freeb[s]), ph ^ 1, tmo, P.status, abort_flag)) break;
+                if (lane == 0) {
+                    const uint32_t fb = smem_addr(&fullb[s]);
+                    const int kc = kc0 + i;
+                    if (weights) {
+                        uint8_t* ws = wsm + s * C::kWSlot;
+                        int srows = 0, sgrp0 = 0;
+                        if (C::kSBytes > 0) {
+                            sgrp0 = (kc * kKC) / P.g;
+                            srows = (P.g >= kKC) ? 1 : min(kKC / P.g, P.G - sgrp0);
+                        }
+                        mbar_arrive_expect_tx(fb, kWStage + srows * srow_bytes);
+                        bulk_g2s(smem_addr(ws), wsrc + static_cast<size_t>(i) * kWStage, kWStage, fb);
+                        for (int h = 0; h < srows; ++h)
+                            bulk_g2s(smem_addr(ws + kWStage + h * 256), ssrc + static_cast<size_t>(sgrp0 + h) * P.N + n0,
+                                     srow_bytes, fb);
+                        if (i < 8) W4A16_TRACE_AT(4 + i);
+                    } else {
+                        uint8_t* st = smem + s * C::kStage;
+                        mbar_arrive_expect_tx(fb, C::kBBytes);
+                        if (C::kIsMsd) {
 #pragma unroll
-                    for (int r = 0; r < 3; ++r)
-                        tma_load_2d(smem_addr(st + r * TT * 128), &tmap, kc * kKC, r * P.M + tc.t0, fb);
-                } else {
-                    for (int h = 0; h < srows; ++h)
-                        bulk_g2s(smem_addr(st + C::kBBytes + kWStage + h * 256),
-                                 ssrc + static_cast<size_t>(sgrp0 + h) * P.N + n0, srow_bytes, fb);
-                    tma_load_2d(smem_addr(st), &tmap, kc * kKC, tc.t0, fb);
-                    tma_load_2d(smem_addr(st + TT * 128), &tmap, kc * kKC + 64, tc.t0, fb);
+                            for (int r = 0; r < 3; ++r)
+                                tma_load_2d(smem_addr(st + r * TT * 128), &tmap, kc * kKC, r * P.M + tc.t0, fb);
+                        } else {
+                            tma_load_2d(smem_addr(st), &tmap, kc * kKC, tc.t0, fb);
+                            tma_load_2d(smem_addr(st + TT * 128), &tmap, kc * kKC + 64, tc.t0, fb);
+                        }
+                        if (i == 0) W4A16_TRACE_AT(3);
+                    }
                 }
+                __syncwarp();
                 ++issued;
             }
             // Drain: every copy issued has landed before the CTA may exit.
-            for (int s = 0; s < LS && s < issued; ++s) {
-                const int last = s + ((issued - 1 - s) / LS) * LS;
-                mbar_wait(smem_addr(&full_bar[s]), (last / LS) & 1, tmo, P.status, nullptr);
+            for (int s = 0; s < ring && s < issued; ++s) {
+                const int last = s + ((issued - 1 - s) / ring) * ring;
+                mbar_wait(smem_addr(&fullb[s]), (last / ring) & 1, tmo, P.status, nullptr);
             }
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ============================ MMA issuer ============================
-        if (lane == 0) {
+    } else if (warp >= 2 && warp < 2 + C::kMaxIssuers) {
+        // ============================ MMA issuers ============================
+        // Issuer q takes chunks q, q + issuers, ...; it waits for the chunk's
+        // A operand (converter) and activation tile (producer), and one commit
+        // per chunk frees the operand stage for both.  The warp runs
+        // converged; lane 0 issues the MMAs and commits.
+        const int q = warp - 2;
+        if (q < issuers) {
             constexpr uint32_t idesc = C::kIsMsd ? idesc_s8_s32(C::kMmaN) : idesc_f16_f32(C::kMmaN);
-            int ab = 0;
-            uint32_t abph = 0;
-            for (int i = 0; i < nchunks; ++i) {
-                const int s = i % LS;
-                const uint32_t ph = (i / LS) & 1;
-                const int as = i % AS;
-                const uint32_t aph = (i / AS) & 1;
-                if (!mbar_wait(smem_addr(&full_bar[s]), ph, tmo, P.status, abort_flag)) break;
-                if (!mbar_wait(smem_addr(&afull_bar[as]), aph, tmo, P.status, abort_flag)) break;
+            constexpr int kSteps = C::kIsMsd ? 4 : 8;         // MMA K steps per 128-deep chunk
+            constexpr int kStepK = kKC / kSteps;
+            // group bookkeeping without divisions in the step loop: K steps
+            // per group (g is a multiple of 32, so of kStepK), as a shift when
+            // it is a power of two
+            const int gsteps = P.g / kStepK;
+            const bool gpow2 = (gsteps & (gsteps - 1)) == 0;
+            const int gshift = __ffs(gsteps) - 1;
+            bool first_chunk = true;
+            for (int i = q; i < nchunks; i += issuers) {
+                const int s = i % ST;
+                const uint32_t ph = (i / ST) & 1;
+                if (i == 2) W4A16_TRACE_AT(57);
+                if (!mbar_wait(smem_addr(&afull_bar[s]), ph, tmo, P.status, abort_flag)) break;
+                if (!mbar_wait(smem_addr(&bfull_bar[s]), ph, tmo, P.status, abort_flag)) break;
+                if (i == 2) W4A16_TRACE_AT(58);
                 tc_fence_after();
-                const uint32_t b_base = smem_addr(smem + s * C::kStage);
-                const uint32_t a_base = tmem_a0 + as * C::kACols;
+                const uint64_t bdesc = smem_desc_sw128(smem_addr(smem + s * C::kStage));
+                const uint32_t a_base = tmem_a0 + s * C::kACols;
                 const int kc = kc0 + i;
+                const int nsteps = min(kSteps, (P.K - kc * kKC) / kStepK);   // K-padding steps are skipped
+                const int step0 = i * kSteps;        // K step index from the split's first group boundary
                 bool failed = false;
-                if (C::kIsMsd) {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int kg = kc * kKC + 32 * j;
-                        if (kg >= P.K) break;
-                        const bool first = (kg % P.g) == 0;
-                        const bool last = ((kg + 32) % P.g) == 0;
-                        if (first) {
-                            if (!mbar_wait(smem_addr(&accempty_bar[ab]), abph ^ 1, tmo, P.status, abort_flag)) {
+                for (int j = 0; j < kSteps; ++j) {
+                    if (j >= nsteps) break;
+                    // B operand: 32-byte K steps inside the 128-byte swizzle row;
+                    // DEQUANT's chunk spans two 64-wide atoms of TT rows each
+                    const uint64_t bd = C::kIsMsd ? bdesc + 2 * j : bdesc + ((j >> 2) * (TT * 128) >> 4) + 2 * (j & 3);
+                    if (C::kGroupAcc) {
+                        const int st_ = step0 + j;
+                        const int grel = gpow2 ? (st_ >> gshift) : (st_ / gsteps);     // group within the split
+                        const int gpos = st_ - grel * gsteps;                          // step within the group
+                        const int ab = (grp0 + grel) % C::kNBuf;
+                        if (gpos == 0) {
+                            // the epilogue has read this buffer (MSD: and reset it to the bias)
+                            if (!mbar_wait(smem_addr(&accempty_bar[ab]), (grel / C::kNBuf) & 1, tmo, P.status,
+                                           abort_flag)) {
                                 failed = true;
                                 break;
                             }
+                            if (i == 2) W4A16_TRACE_AT(59);
                             tc_fence_after();
                         }
-                        mma_i8_ts(tmem + ab * C::kAccStride, a_base + 8 * j, smem_desc_sw128(b_base + 32 * j), idesc,
-                                  first ? 0u : 1u);
-                        if (last) {
-                            tc_commit(smem_addr(&accfull_bar[ab]));
-                            ab ^= 1;
-                            if (ab == 0) abph ^= 1;
+                        const uint32_t d = tmem + ab * C::kAccStride;
+                        if (lane == 0) {
+                            if (C::kIsMsd) mma_i8_ts(d, a_base + 8 * j, bd, idesc, 1u);
+                            else mma_f16_ts(d, a_base + 8 * j, bd, idesc, gpos == 0 ? 0u : 1u);
+                            if (i == 2 && j < 4) W4A16_TRACE_AT(60 + j);
+                            if (gpos == gsteps - 1) tc_commit(smem_addr(&accfull_bar[ab]));
                         }
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const int kg = kc * kKC + 16 * j;
-                        if (kg >= P.K) break;
-                        const uint32_t boff = (j >> 2) * (TT * 128) + (j & 3) * 32;
-                        mma_f16_ts(tmem, a_base + 8 * j, smem_desc_sw128(b_base + boff), idesc,
-                                   (i > 0 || j > 0) ? 1u : 0u);
+                        __syncwarp();
+                    } else {
+                        if (lane == 0) mma_f16_ts(tmem, a_base + 8 * j, bd, idesc, (first_chunk && j == 0) ? 0u : 1u);
+                        __syncwarp();
                     }
                 }
-                tc_commit(smem_addr(&empty_bar[s]));
-                tc_commit(smem_addr(&aempty_bar[as]));
+                if (lane == 0) {
+                    if (i < 8) W4A16_TRACE_AT(28 + i);
+                    tc_commit(smem_addr(&sfree_bar[s]));
+                }
+                __syncwarp();
+                first_chunk = false;
                 if (failed) break;
-                if (!C::kIsMsd && i == nchunks - 1) tc_commit(smem_addr(&accfull_bar[0]));
             }
-            // Every MMA issued has completed before Tensor Memory is freed.
-            tc_commit(smem_addr(done_bar));
-            mbar_wait(smem_addr(done_bar), 0, tmo, P.status, nullptr);
+            if (lane == 0) {
+                if (!C::kGroupAcc) tc_commit(smem_addr(&accfull_bar[0]));
+                // Every MMA issued has completed before Tensor Memory is freed.
+                tc_commit(smem_addr(&done_bar[q]));
+            }
+            __syncwarp();
+            mbar_wait(smem_addr(&done_bar[q]), 0, tmo, P.status, nullptr);
         }
         __syncwarp();
-    } else if (warp < 6) {
+    } else if (warp >= C::kConvWarp0 && warp < C::kEpiWarp0) {
         // ============================ converters ============================
+        // Group cg takes chunks cg, cg + NCONV, ...: packed weights from the
+        // weight ring -> registers -> the MMA A operand in Tensor Memory.
+        const int cg = (warp - C::kConvWarp0) >> 2;            // converter group
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32);
         const int r = lane_base + lane;                        // weight row in the tile
-        for (int i = 0; i < nchunks; ++i) {
-            const int s = i % LS;
-            const uint32_t ph = (i / LS) & 1;
-            const int as = i % AS;
-            const uint32_t aph = (i / AS) & 1;
-            if (!mbar_wait(smem_addr(&full_bar[s]), ph, tmo, P.status, abort_flag)) break;
-            if (!mbar_wait(smem_addr(&aempty_bar[as]), aph ^ 1, tmo, P.status, abort_flag)) break;
-            tc_fence_after();
-            const uint8_t* st = smem + s * C::kStage;
-            const uint8_t* wst = st + C::kBBytes;
+        for (int i = cg; i < nchunks; i += NCONV) {
+            const int s = i % ST;
+            const uint32_t ph = (i / ST) & 1;
+            const int w = i % WST;
+            const uint32_t wph = (i / WST) & 1;
+            if (!mbar_wait(smem_addr(&wfull_bar[w]), wph, tmo, P.status, abort_flag)) break;
+            if (cg == 0 && (warp & 3) == 0 && lane == 0 && i < 8) W4A16_TRACE_AT(12 + i);
+            const uint8_t* wst = wsm + w * C::kWSlot;
             uint4 q[4];
 #pragma unroll
             for (int p = 0; p < 4; ++p) q[p] = *reinterpret_cast<const uint4*>(wst + p * 2048 + r * 16);
-            const uint32_t a_addr = tmem_a0 + as * C::kACols + (lane_base << 16);
-            if (C::kIsMsd) {
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_addr(&empty_bar[s]));
+            __half sv[4];
+            if (!C::kIsMsd && !SEPI) {
+                const __half* sst = reinterpret_cast<const __half*>(wst + kWStage);
+                const int kc = kc0 + i;
+                const int sgrp0 = (kc * kKC) / P.g;
 #pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const int row = (P.g >= kKC) ? 0 : ((kc * kKC + 32 * p) / P.g - sgrp0);
+                    sv[p] = sst[row * kBN + r];
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&wempty_bar[w]));      // weight slot read
+            // the A operand columns of stage s are free once the MMA of the
+            // stage's previous chunk has completed
+            if (!mbar_wait(smem_addr(&sfree_bar[s]), ph ^ 1, tmo, P.status, abort_flag)) break;
+            tc_fence_after();
+            const uint32_t a_addr = tmem_a0 + s * C::kACols + (lane_base << 16);
+            if (C::kIsMsd) {
+W4A16_ROLE_UNROLL
                 for (int p = 0; p < 4; ++p) {
                     uint32_t o[8];
                     int8_word(q[p].x, o + 0);
@@ -471,156 +624,234 @@ __global__ void __launch_bounds__(kThreads, MINB)
                     int8_word(q[p].w, o + 6);
                     tmem_st8(a_addr + 8 * p, o);
                 }
-            } else {
-                const __half* sst = reinterpret_cast<const __half*>(st + C::kBBytes + kWStage);
-                const int kc = kc0 + i;
-                const int sgrp0 = (kc * kKC) / P.g;
-                __half sv[4];
-#pragma unroll
+            } else if (SEPI) {
+W4A16_ROLE_UNROLL
                 for (int p = 0; p < 4; ++p) {
-                    const int row = (P.g >= kKC) ? 0 : ((kc * kKC + 32 * p) / P.g - sgrp0);
-                    sv[p] = sst[row * kBN + r];
+                    uint32_t o[16];
+                    int4_to_half2x4(q[p].x, o + 0);
+                    int4_to_half2x4(q[p].y, o + 4);
+                    int4_to_half2x4(q[p].z, o + 8);
+                    int4_to_half2x4(q[p].w, o + 12);
+                    tmem_st16(a_addr + 16 * p, o);
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_addr(&empty_bar[s]));
-#pragma unroll
+            } else {
+W4A16_ROLE_UNROLL
                 for (int p = 0; p < 4; ++p) {
                     const __half2 s2 = __halves2half2(sv[p], sv[p]);
                     uint32_t o[16];
-                    dequant_word(q[p].x, s2, o + 0);
-                    dequant_word(q[p].y, s2, o + 4);
-                    dequant_word(q[p].z, s2, o + 8);
-                    dequant_word(q[p].w, s2, o + 12);
+                    int4_to_half2x4_scaled(q[p].x, s2, o + 0);
+                    int4_to_half2x4_scaled(q[p].y, s2, o + 4);
+                    int4_to_half2x4_scaled(q[p].z, s2, o + 8);
+                    int4_to_half2x4_scaled(q[p].w, s2, o + 12);
                     tmem_st16(a_addr + 16 * p, o);
                 }
             }
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&afull_bar[as]));
+            if (lane == 0) mbar_arrive(smem_addr(&afull_bar[s]));
+            if (cg == 0 && (warp & 3) == 0 && lane == 0 && i < 8) W4A16_TRACE_AT(20 + i);
         }
-    } else {
+    } else if (warp >= C::kEpiWarp0) {
         // ============================ epilogue ============================
+        const int eg = (warp - C::kEpiWarp0) >> 2;             // epilogue group: a slice of the tokens
+        const int et = threadIdx.x - 32 * C::kEpiWarp0;        // 0 .. kEpiThreads-1
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32);
         const int r = lane_base + lane;
         const int n = n0 + r;
         const bool n_ok = n < P.N;
         const int nt = tc.t_end - tc.t0;
+        constexpr int TE = C::kTokPerEpi;
+        const int tb = eg * TE;                                 // first token of this group
         const uint32_t t_addr = tmem + (lane_base << 16);
+        float acc[TE];
+#pragma unroll
+        for (int t = 0; t < TE; ++t) acc[t] = 0.f;
+        bool ok = true;
 
-        if (C::kIsMsd) {
-            float acc[TT];
+        if (C::kGroupAcc) {
+            if (C::kIsMsd) {
+                // every accumulator buffer starts at the bias
 #pragma unroll
-            for (int t = 0; t < TT; ++t) acc[t] = 0.f;
-            const int grp0 = (kc0 * kKC) / P.g;
-            const int grp1 = min(kc1 * kKC, P.K) / P.g;
+                for (int b = 0; b < C::kNBuf; ++b)
+#pragma unroll
+                    for (int rr = 0; rr < 3; ++rr)
+#pragma unroll
+                        for (int c = 0; c < TE / 8; ++c)
+                            tmem_st8_fill(t_addr + b * C::kAccStride + rr * TT + tb + 8 * c, kAccBiasBits);
+                tmem_st_wait();
+                tc_fence_before();
+            }
+            __syncwarp();
+            if (lane == 0)          // release every buffer to the MMA
+                for (int b = 0; b < C::kNBuf; ++b) mbar_arrive(smem_addr(&accempty_bar[b]));
+            griddep_wait();    // A_max comes from the expansion kernel; y is shared with earlier kernels
+            if (warp == C::kEpiWarp0 && lane == 0) W4A16_TRACE_AT(52);
+
+            const int ngroups = min(kc1 * kKC, P.K) / P.g - grp0;
             const __half* sc_e = P.scale[tc.e];
-            bool ok = true;
-            for (int j = 0; j < grp1 - grp0; ++j) {
+            float am_next = 0.f, sc_next = 0.f;
+            if (ngroups > 0) {
+                if (C::kIsMsd && et < nt) am_next = __ldg(P.amax + static_cast<size_t>(grp0) * P.M + tc.t0 + et);
+                if (n_ok && sc_e) sc_next = __half2float(sc_e[static_cast<size_t>(grp0) * P.N + n]);
+            }
+            for (int j = 0; j < ngroups; ++j) {
                 const int grp = grp0 + j;
-                const int ab = j & 1;
-                const uint32_t abph = (j >> 1) & 1;
-                const float sc = (n_ok && sc_e) ? __half2float(sc_e[static_cast<size_t>(grp) * P.N + n]) : 0.f;
-                const float* am_row = P.amax + static_cast<size_t>(grp) * P.M + tc.t0;
-                if (!mbar_wait(smem_addr(&accfull_bar[ab]), abph, tmo, P.status, abort_flag)) {
-                    ok = false;
-                    break;
+                const int ab = grp % C::kNBuf;
+                const uint32_t abph = (j / C::kNBuf) & 1;
+                float* am_slot = amax_sm + (j & 1) * TT;
+                if (C::kIsMsd && et < TT) am_slot[et] = am_next;
+                const float sc = sc_next;
+                if (j + 1 < ngroups) {           // prefetch the next group's A_max and scale
+                    if (C::kIsMsd)
+                        am_next = (et < nt) ? __ldg(P.amax + static_cast<size_t>(grp + 1) * P.M + tc.t0 + et) : 0.f;
+                    if (n_ok && sc_e) sc_next = __half2float(sc_e[static_cast<size_t>(grp + 1) * P.N + n]);
                 }
+                if (C::kIsMsd) named_bar_sync(1, C::kEpiThreads);   // every epilogue thread, every group
+                if (ok && !mbar_wait(smem_addr(&accfull_bar[ab]), abph, tmo, P.status, abort_flag)) ok = false;
+                if (!ok) continue;
+                if (warp == C::kEpiWarp0 && lane == 0 && j < 8) W4A16_TRACE_AT(36 + j);
                 tc_fence_after();
-                const uint32_t b_addr = t_addr + ab * C::kAccStride;
+                const uint32_t b_addr = t_addr + ab * C::kAccStride + tb;
+                if (C::kIsMsd) {
+                    const float scc = sc * kC1;
 #pragma unroll
-                for (int c = 0; c < TT / 16; ++c) {
-                    uint32_t y1[16], y2[16], y3[16];
-                    tmem_ld16(b_addr + 16 * c, y1);
-                    tmem_ld16(b_addr + TT + 16 * c, y2);
-                    tmem_ld16(b_addr + 2 * TT + 16 * c, y3);
-                    tmem_ld_wait();
+                    for (int c = 0; c < TE / 8; ++c) {
+                        uint32_t y1[8], y2[8], y3[8];
+                        tmem_ld8(b_addr + 8 * c, y1);
+                        tmem_ld8(b_addr + TT + 8 * c, y2);
+                        tmem_ld8(b_addr + 2 * TT + 8 * c, y3);
+                        const float4 a0 = reinterpret_cast<const float4*>(am_slot + tb + 8 * c)[0];
+                        const float4 a1 = reinterpret_cast<const float4*>(am_slot + tb + 8 * c)[1];
+                        const float am[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const int t = 16 * c + q;
-                        const float am = (t < nt) ? __ldg(am_row + t) : 0.f;
-                        // equation 10, then equation 11's running sum
-                        const float v = fmaf(static_cast<float>(static_cast<int32_t>(y3[q])), kC3,
-                                             fmaf(static_cast<float>(static_cast<int32_t>(y2[q])), kC2,
-                                                  static_cast<float>(static_cast<int32_t>(y1[q])) * kC1));
-                        acc[t] = fmaf(v, am * sc, acc[t]);
-                    }
-                    if (P.dbg_yint != nullptr && n_ok && n >= P.dbg_n0 && n < P.dbg_n1) {
-                        const int wn = P.dbg_n1 - P.dbg_n0, wm = P.dbg_m1 - P.dbg_m0;
-                        const size_t plane = static_cast<size_t>(wm) * P.G * wn;
+                        for (int qq = 0; qq < 8; ++qq) {
+                            // exact Y_i as floats, then equation 10 and equation 11's running sum
+                            const float d1 = __uint_as_float(y1[qq]) - kAccBias;
+                            const float d2 = __uint_as_float(y2[qq]) - kAccBias;
+                            const float d3 = __uint_as_float(y3[qq]) - kAccBias;
+                            const float v = fmaf(d3, kR3, fmaf(d2, kR2, d1));
+                            acc[8 * c + qq] = fmaf(v, am[qq] * scc, acc[8 * c + qq]);
+                        }
+                        if (DBG && n_ok && n >= P.dbg_n0 && n < P.dbg_n1) {
+                            const int wn = P.dbg_n1 - P.dbg_n0, wm = P.dbg_m1 - P.dbg_m0;
+                            const size_t plane = static_cast<size_t>(wm) * P.G * wn;
 #pragma unroll
-                        for (int q = 0; q < 16; ++q) {
-                            const int m = tc.t0 + 16 * c + q;
-                            if (16 * c + q < nt && m >= P.dbg_m0 && m < P.dbg_m1) {
-                                const size_t o = (static_cast<size_t>(m - P.dbg_m0) * P.G + grp) * wn + (n - P.dbg_n0);
-                                P.dbg_yint[o] = static_cast<int32_t>(y1[q]);
-                                P.dbg_yint[plane + o] = static_cast<int32_t>(y2[q]);
-                                P.dbg_yint[2 * plane + o] = static_cast<int32_t>(y3[q]);
-                                if (n == P.dbg_n0)
-                                    P.dbg_amax[static_cast<size_t>(m - P.dbg_m0) * P.G + grp] = __ldg(am_row + 16 * c + q);
+                            for (int qq = 0; qq < 8; ++qq) {
+                                const int t = tb + 8 * c + qq;
+                                const int m = tc.t0 + t;
+                                if (t < nt && m >= P.dbg_m0 && m < P.dbg_m1) {
+                                    const size_t o = (static_cast<size_t>(m - P.dbg_m0) * P.G + grp) * wn + (n - P.dbg_n0);
+                                    P.dbg_yint[o] = static_cast<int32_t>(y1[qq] - kAccBiasBits);
+                                    P.dbg_yint[plane + o] = static_cast<int32_t>(y2[qq] - kAccBiasBits);
+                                    P.dbg_yint[2 * plane + o] = static_cast<int32_t>(y3[qq] - kAccBiasBits);
+                                    if (n == P.dbg_n0)
+                                        P.dbg_amax[static_cast<size_t>(m - P.dbg_m0) * P.G + grp] = am[qq];
+                                }
                             }
                         }
+                    }
+                    // reset this group's columns to the bias
+#pragma unroll
+                    for (int rr = 0; rr < 3; ++rr)
+#pragma unroll
+                        for (int c = 0; c < TE / 8; ++c) tmem_st8_fill(b_addr + rr * TT + 8 * c, kAccBiasBits);
+                    tmem_st_wait();
+                } else {
+#pragma unroll
+                    for (int c = 0; c < TE / 16; ++c) {
+                        uint32_t v[16];
+                        tmem_ld16(b_addr + 16 * c, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) acc[16 * c + k] = fmaf(__uint_as_float(v[k]), sc, acc[16 * c + k]);
                     }
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_addr(&accempty_bar[ab]));
+                if (warp == C::kEpiWarp0 && lane == 0 && j < 8) W4A16_TRACE_AT(44 + j);
             }
-            if (ok && n_ok) {
+            if (ok && P.splits == 1 && P.write_y && n_ok) {
 #pragma unroll
-                for (int t = 0; t < TT; ++t)
-                    if (t < nt) emit_value(P, tc, n, t, acc[t]);
+                for (int t = 0; t < TE; ++t)
+                    if (tb + t < nt) P.y[static_cast<size_t>(tc.t0 + tb + t) * P.N + n] = __float2half_rn(acc[t]);
             }
-        } else if (nchunks > 0) {
-            if (mbar_wait(smem_addr(&accfull_bar[0]), 0, tmo, P.status, abort_flag)) {
+        } else {
+            // one accumulator over all of K (scales applied by the converter)
+            griddep_wait();
+            ok = nchunks > 0 && mbar_wait(smem_addr(&accfull_bar[0]), 0, tmo, P.status, abort_flag);
+            if (ok) {
+                if (warp == C::kEpiWarp0 && lane == 0) W4A16_TRACE_AT(36);
                 tc_fence_after();
 #pragma unroll 1
-                for (int c = 0; c < TT / 16; ++c) {
-                    uint32_t v[16];
-                    tmem_ld16(t_addr + 16 * c, v);
+                for (int c = 0; c < TE / 16; ++c) {
+                    uint32_t u[16];
+                    tmem_ld16(t_addr + tb + 16 * c, u);
                     tmem_ld_wait();
-                    if (n_ok) {
+                    if (P.write_y && n_ok) {
 #pragma unroll
-                        for (int q = 0; q < 16; ++q)
-                            if (16 * c + q < nt) emit_value(P, tc, n, 16 * c + q, __uint_as_float(v[q]));
+                        for (int k = 0; k < 16; ++k)
+                            if (tb + 16 * c + k < nt)
+                                P.y[static_cast<size_t>(tc.t0 + tb + 16 * c + k) * P.N + n] =
+                                    __float2half_rn(__uint_as_float(u[k]));
                     }
                 }
                 tc_fence_before();
             }
         }
 
-        // Split-K: the last CTA of this (token tile, column tile) to arrive
-        // adds the partial sums in split order (deterministic) and stores y.
-        if (P.splits > 1) {
-            __threadfence();
-            named_bar_sync(1, 128);          // every epilogue thread reaches this
-            if (r == 0) {
-                int last = 0;
-                if (!*abort_flag) {
-                    const uint32_t tile = blockIdx.z * P.n_tiles + blockIdx.x;
-                    const uint32_t old = atomicAdd(&P.counters[tile], 1u);
-                    last = (old == static_cast<uint32_t>(P.splits - 1)) ? 1 : 0;
-                }
-                *last_flag = last;
-            }
-            named_bar_sync(1, 128);
-            if (*last_flag) {
-                __threadfence();
-                if (n_ok && P.write_y) {
-                    for (int t = 0; t < nt; ++t) {
-                        float sum = 0.f;
-                        for (int sp = 0; sp < P.splits; ++sp)
-                            sum += __ldcg(&P.partial[(static_cast<size_t>(sp) * P.M + tc.t0 + t) * P.N + n]);
-                        P.y[static_cast<size_t>(tc.t0 + t) * P.N + n] = __float2half_rn(sum);
-                    }
-                }
-                if (r == 0) P.counters[blockIdx.z * P.n_tiles + blockIdx.x] = 0;
+        // Split-K (decode tile only): push this CTA's partial sums into the
+        // reduction buffer of the cluster rank that owns them: element
+        // e = t * 128 + r belongs to rank e / per and lands in slot
+        // [this rank][e - owner * per] there.
+        if (C::kRedBytes > 0 && P.splits > 1 && ok) {
+            const int S = P.splits;
+            const int per = (TT * kBN + S - 1) / S;
+            const uint32_t me = cluster_ctarank();
+            const uint32_t red_base = smem_addr(red);
+#pragma unroll
+            for (int t = 0; t < TE; ++t) {
+                const int e = (tb + t) * kBN + r;
+                const int owner = e / per;
+                st_cluster_f32(map_to_rank(red_base + 4u * static_cast<uint32_t>(me * per + (e - owner * per)),
+                                           static_cast<uint32_t>(owner)),
+                               acc[t]);
             }
         }
     }
 
+    // Split-K: one cluster barrier (every thread of every CTA) makes all
+    // pushed partials visible; each rank then adds, in rank order
+    // (deterministic), the S partials of the elements it owns and stores y.
+    // After the barrier no CTA touches another's shared memory.
+    if (C::kRedBytes > 0 && P.splits > 1) {
+        __syncwarp();
+        if (warp == C::kEpiWarp0 && lane == 0) W4A16_TRACE_AT(53);
+        cluster_sync_all();
+        if (warp == C::kEpiWarp0 && lane == 0) W4A16_TRACE_AT(54);
+        if (warp >= C::kEpiWarp0 && P.write_y && !*abort_flag) {
+            const int S = P.splits;
+            const int per = (TT * kBN + S - 1) / S;
+            const int me = static_cast<int>(cluster_ctarank());
+            const int nt = tc.t_end - tc.t0;
+            for (int el = threadIdx.x - 32 * C::kEpiWarp0; el < per; el += C::kEpiThreads) {
+                const int e = me * per + el;
+                const int t = e / kBN;
+                const int nn = n0 + (e % kBN);
+                if (t >= nt || nn >= P.N) continue;
+                float sum = 0.f;
+                for (int sp = 0; sp < S; ++sp) sum += red[sp * per + el];
+                P.y[static_cast<size_t>(tc.t0 + t) * P.N + nn] = __float2half_rn(sum);
+            }
+        }
+        if (warp == C::kEpiWarp0 && lane == 0) W4A16_TRACE_AT(55);
+    }
+
     tc_fence_before();
     __syncthreads();
+    if (threadIdx.x == 0) W4A16_TRACE_AT(56);
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
