@@ -118,6 +118,12 @@ def max_over_ranks(value: float, device=None) -> float:
     return float(t.item())
 
 
+def whole_job_gbs(bytes_per_step: int, steps: int, world: int, ms_max: float) -> float:
+    """Whole-job GB/s: the bytes every replica processed in `steps` steps over
+    the slowest rank's timed region (`ms_max`, already the max over ranks)."""
+    return bytes_per_step * steps * world / (ms_max * 1e-3) / 1e9
+
+
 def barrier(device=None):
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
@@ -364,7 +370,7 @@ def run_gpu(args, wl, rank, world, local):
     b = step_bytes(wl)
     bytes_step = 2 * b["total"]
     flops_step = 2 * step_flops(wl)
-    value = bytes_step * args.steps * world / (ms * 1e-3) / 1e9
+    value = whole_job_gbs(bytes_step, args.steps, world, ms)
     hbm, bf16, bf16_sus, peak_kind = load_peaks()
 
     # dominant kernel: the variant with the longer call
