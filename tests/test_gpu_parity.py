@@ -195,6 +195,71 @@ def test_repeat_calls_are_deterministic(cuda_lib):
     torch.cuda.synchronize()
 
 
+# ---------------------------------------------------------------- decode GEMV (M <= 4)
+
+# Shapes for the CUDA-core decode kernel: every group size, ragged N and K,
+# and work splits where many CTAs share one column tile (N small, K long) or
+# one CTA spans two tiles (N large, K short).
+GEMV = [
+    # (M, K, N, g)                       what it covers
+    (1, 4096, 136, 128),                 # 2 tiles x 32 chunks: ~32 CTAs add into each tile
+    (2, 256, 14336, 64),                 # 224 blocks over the SMs: CTAs straddle tile edges
+    (3, 1280, 520, 32),                  # four groups per chunk, ragged N, M below the row template
+    (4, 768, 1032, 256),                 # group spanning two chunks, ragged N
+    (1, 2560, 392, 512),                 # group of 512 (four chunks), K = 5 groups
+    (4, 8192, 264, 128),                 # the largest M * K the kernel takes
+    (2, 96, 128, 32),                    # K shorter than one chunk
+]
+
+
+@pytest.mark.parametrize("M,K,N,g", GEMV)
+def test_gemv_msd(cuda_lib, M, K, N, g):
+    w4 = cuda_lib
+    c = make_case(M, K, N, g, seed=M * 131 + K * 7 + N * 3 + g)
+    c.x[M - 1, :g] = 0                   # an all-zero group
+    dev = upload(w4, c)
+    y = run_dense(w4, w4.OP_MSD, c, dev)
+    assert_msd_close(y, oracle.msd(c.x, c.wp[0], c.scale[0], g), f"gemv msd {M}x{K}x{N} g{g}")
+
+
+@pytest.mark.parametrize("M,K,N,g", GEMV)
+def test_gemv_dequant(cuda_lib, M, K, N, g):
+    w4 = cuda_lib
+    c = make_case(M, K, N, g, seed=M * 137 + K * 5 + N * 11 + g)
+    dev = upload(w4, c)
+    y = run_dense(w4, w4.OP_DEQUANT, c, dev)
+    assert_deq_close(y, oracle.dequant(c.x, c.wp[0], c.scale[0], g), f"gemv dequant {M}x{K}x{N} g{g}")
+
+
+def test_gemv_repeat_calls_are_deterministic(cuda_lib):
+    """The tile counters reset themselves and the partials are added in CTA
+    order, so repeated calls on one workspace give the same bits."""
+    w4 = cuda_lib
+    c = make_case(1, 4096, 1032, 128, seed=77)
+    dev = upload(w4, c)
+    for op in (w4.OP_MSD, w4.OP_DEQUANT):
+        ws = w4.alloc_workspace(op, c.M, c.K, c.N, c.g)
+        ys = [run_dense(w4, op, c, dev, ws) for _ in range(4)]
+        assert all(np.array_equal(ys[0], v) for v in ys[1:])
+
+
+def test_gemv_page_example_distributions(cuda_lib):
+    """The page's own value ranges (x, scale ~ U[-3, 3], w in [-7, 7]) at M = 1."""
+    w4 = cuda_lib
+    rng = np.random.default_rng(4847346)
+    M, K, N, g = 1, 2048, 1536, 128
+    x = rng.uniform(-3, 3, (M, K)).astype(np.float16)
+    w = rng.integers(-7, 8, (K, N), dtype=np.int8)
+    sc = rng.uniform(-3, 3, (K // g, N)).astype(np.float16)
+    c = make_case(M, K, N, g, seed=1)
+    c.x[:] = x
+    c.wp[0] = pack_int4(w)
+    c.scale[0] = sc
+    dev = upload(w4, c)
+    assert_msd_close(run_dense(w4, w4.OP_MSD, c, dev), oracle.msd(c.x, c.wp[0], sc, g), "gemv msd page")
+    assert_deq_close(run_dense(w4, w4.OP_DEQUANT, c, dev), oracle.dequant(c.x, c.wp[0], sc, g), "gemv deq page")
+
+
 # ---------------------------------------------------------------- grouped experts
 
 def test_grouped_small_with_empty_experts(cuda_lib):

@@ -8,8 +8,12 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libw4a16.so")
 SOURCES = [os.path.join(CSRC, "w4a16_api.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("w4a16_kernels.cuh", "sm100_ptx.cuh")] + \
-    [os.path.join(ROOT, "include", "w4a16.h")]
+
+
+def deps():
+    """Every source and header the library is built from."""
+    return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cu", ".cuh", ".h"))) + \
+        [os.path.join(ROOT, "include", "w4a16.h")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -27,7 +31,7 @@ def nvcc() -> str:
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and os.path.exists(LIB):
         t = os.path.getmtime(LIB)
-        if all(os.path.getmtime(d) <= t for d in DEPS):
+        if all(os.path.getmtime(d) <= t for d in deps()):
             return LIB
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [nvcc(), *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []), *SOURCES, "-o", tmp]

@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "../../include/w4a16.h"
+#include "w4a16_gemv.cuh"
 #include "w4a16_kernels.cuh"
 
 using namespace w4a16;
@@ -35,6 +36,7 @@ namespace {
 std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
 
 constexpr size_t kHeaderBytes = 256;   // device status word + padding
+constexpr int kMaxSmemOptin = 227 * 1024;   // dynamic shared memory a CTA may opt in to
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -151,11 +153,36 @@ Shape grouped_shape(int op, int T, int K, int N, int g, int E)
     return s;
 }
 
+// ---------------------------------------------------------------- the CUDA-core decode GEMV
+
+// Largest M that takes the GEMV (w4a16_gemv.cuh) instead of the tensor-core
+// decode tile; W4A16_GEMV_MAX_M overrides it (0 turns the GEMV off).
+int gemv_max_m(int op)
+{
+    static int v[2] = {-1, -1};
+    if (v[op] < 0) {
+        const char* e = std::getenv("W4A16_GEMV_MAX_M");
+        int d = 4;
+        if (e && *e) d = std::atoi(e);
+        v[op] = std::max(0, std::min(d, 4));
+    }
+    return v[op];
+}
+
+bool use_gemv(int op, int M, int K, int E)
+{
+    return E == 1 && M >= 1 && M <= gemv_max_m(op) && static_cast<long long>(M) * K <= kGemvMaxMK;
+}
+
+// CTAs of the GEMV: one per SM at most, never more than there are 32-column
+// blocks.
+int gemv_ctas(int nblk) { return std::min(nblk, sm_count()); }
+
 struct WsLayout {
-    size_t xq = 0, amax = 0, total = 0;
+    size_t xq = 0, amax = 0, rec = 0, rec_amax = 0, total = 0;
 };
 
-WsLayout ws_layout(int op, const Shape& s, int M, int K, int N, int g)
+WsLayout ws_layout(int op, const Shape& s, int M, int K, int N, int g, int E = 1)
 {
     (void)s;
     (void)N;
@@ -166,6 +193,13 @@ WsLayout ws_layout(int op, const Shape& s, int M, int K, int N, int g)
         off += align256(static_cast<size_t>(3) * M * K);
         L.amax = off;
         off += align256(static_cast<size_t>(K / g) * M * 4);
+        if (use_gemv(op, M, K, E)) {
+            // the decode GEMV's digit records [K/32][M][28 words] and A_max [M][K/g]
+            L.rec = off;
+            off += align256(static_cast<size_t>(K / 32) * M * kGemvRecWords * 4);
+            L.rec_amax = off;
+            off += align256(static_cast<size_t>(K / g) * M * 4);
+        }
     }
     L.total = off;
     return L;
@@ -319,6 +353,99 @@ void base_params(GemmParams& P, int M, int K, int N, int g, const Shape& s, void
     P.write_y = 1;
 }
 
+template <int VAR, int MR>
+w4a16_status launch_gemv_mr(const GemvParams& P, cudaStream_t stream)
+{
+    using C = GemvCfg<VAR, MR>;
+    auto kern = gemv_kernel<VAR, MR>;
+    const int smem = C::smem_bytes(P.M, P.K);
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [&] {
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmemOptin);
+    });
+    if (attr_err != cudaSuccess) return W4A16_ERR_CUDA;
+    if (smem > kMaxSmemOptin) return W4A16_ERR_UNSUPPORTED;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(P.ctas), 1, 1);
+    cfg.blockDim = dim3(kGemvThreads, 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = use_pdl() ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, kern, P) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return W4A16_ERR_CUDA;
+    }
+    return W4A16_OK;
+}
+
+template <int NSUB>
+cudaError_t launch_gemv_expand_n(const __half* x, int M, int K, int g, uint32_t* rec, float* amax, cudaStream_t s)
+{
+    const int span = NSUB * kKC;
+    const long long warps = static_cast<long long>(M) * ((K + span - 1) / span);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((warps + 7) / 8), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = use_pdl() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, gemv_expand_kernel<NSUB>, x, M, K, g, rec, amax);
+}
+
+w4a16_status launch_gemv(int op, const void* x, const void* w_packed, const void* scale, int M, int K, int N, int g,
+                         void* y, void* ws, const Shape& s, const WsLayout& L, cudaStream_t stream)
+{
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    GemvParams P;
+    std::memset(&P, 0, sizeof(P));
+    P.x = static_cast<const __half*>(x);
+    P.w = static_cast<const uint8_t*>(w_packed);
+    P.scale = static_cast<const __half*>(scale);
+    P.y = static_cast<__half*>(y);
+    P.M = M;
+    P.K = K;
+    P.N = N;
+    P.g = g;
+    P.G = K / g;
+    P.kchunks = s.kchunks;
+    P.npieces = K / 32;
+    P.nblk = cdiv(N, 32);
+    P.ctas = gemv_ctas(P.nblk);
+    if (op == W4A16_OP_MSD) {
+        uint32_t* rec = reinterpret_cast<uint32_t*>(wsb + L.rec);
+        float* amax = reinterpret_cast<float*>(wsb + L.rec_amax);
+        P.rec = rec;
+        P.amax = amax;
+        const __half* xh = static_cast<const __half*>(x);
+        cudaError_t e;
+        switch (std::max(1, g / kKC)) {
+            case 1: e = launch_gemv_expand_n<1>(xh, M, K, g, rec, amax, stream); break;
+            case 2: e = launch_gemv_expand_n<2>(xh, M, K, g, rec, amax, stream); break;
+            case 3: e = launch_gemv_expand_n<3>(xh, M, K, g, rec, amax, stream); break;
+            case 4: e = launch_gemv_expand_n<4>(xh, M, K, g, rec, amax, stream); break;
+            default: return W4A16_ERR_UNSUPPORTED;
+        }
+        if (e != cudaSuccess) {
+            (void)cudaGetLastError();
+            return W4A16_ERR_CUDA;
+        }
+        if (M == 1) return launch_gemv_mr<kMsd, 1>(P, stream);
+        if (M == 2) return launch_gemv_mr<kMsd, 2>(P, stream);
+        return launch_gemv_mr<kMsd, 4>(P, stream);
+    }
+    if (M == 1) return launch_gemv_mr<kDeq, 1>(P, stream);
+    if (M == 2) return launch_gemv_mr<kDeq, 2>(P, stream);
+    return launch_gemv_mr<kDeq, 4>(P, stream);
+}
+
 // Shared body of the dense MSD / DEQUANT calls and the debug window.
 w4a16_status dense_matmul(int op, const void* x, const void* w_packed, const void* scale, int M, int K, int N,
                           int g, void* y, void* ws, size_t ws_bytes, cudaStream_t stream, int32_t* dbg_yint,
@@ -354,6 +481,7 @@ w4a16_status dense_matmul(int op, const void* x, const void* w_packed, const voi
         P.dbg_n0 = n0;
         P.dbg_n1 = n1;
     }
+    if (!debug && use_gemv(op, M, K, 1)) return launch_gemv(op, x, w_packed, scale, M, K, N, g, y, ws, s, L, stream);
     CUtensorMap map;
     if (op == W4A16_OP_MSD) {
         int8_t* xq = reinterpret_cast<int8_t*>(wsb + L.xq);
@@ -433,7 +561,7 @@ w4a16_status w4a16_workspace_size(int op, int M, int K, int N, int group_size, i
     if (st != W4A16_OK) return st;
     if (op == W4A16_OP_MSD && group_size > kMaxGroupMsd) return W4A16_ERR_UNSUPPORTED;
     const Shape s = (E == 1) ? dense_shape(op, M, K, N, group_size) : grouped_shape(op, M, K, N, group_size, E);
-    *bytes = ws_layout(op, s, M, K, N, group_size).total;
+    *bytes = ws_layout(op, s, M, K, N, group_size, E).total;
     return W4A16_OK;
 }
 
@@ -492,7 +620,7 @@ w4a16_status w4a16_grouped_matmul(int op, const void* x, const void* const* w_pa
         if (!w_packed[e] || !scale[e] || !aligned16(w_packed[e]) || !aligned16(scale[e]))
             return W4A16_ERR_INVALID_ARG;
     const Shape s = grouped_shape(op, T, K, N, group_size, E);
-    const WsLayout L = ws_layout(op, s, T, K, N, group_size);
+    const WsLayout L = ws_layout(op, s, T, K, N, group_size, E);
     if (workspace_bytes < L.total) return W4A16_ERR_WORKSPACE;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
 

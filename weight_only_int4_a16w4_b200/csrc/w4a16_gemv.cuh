@@ -1,0 +1,406 @@
+// w4a16_gemv.cuh -- the decode kernel for the smallest batches (M <= 4):
+// a GEMV on the CUDA cores, both variants.
+//
+// Operator: y = x . (antiquant_scale (.) W), "WeightQuantBatchMatmulExperiment
+// 算子深度解析" (bjdmk.com.cn/news/4847346), section 4.1 (MSD, steps 1-11)
+// and the plain dequant definition.  At M <= 4 the matmul is a stream of
+// weights with a handful of multiply-adds per weight: a 128 x 16 tensor-core
+// tile would be mostly padding, so the CUDA cores do the arithmetic and the
+// kernel is shaped around getting every weight byte in flight at once.
+//
+// Work split: output columns only.  The columns form blocks of 32 (one warp
+// width); CTA c of P takes blocks [c*B/P, (c+1)*B/P) and all of K, so no
+// partial sums leave the CTA.  Inside a CTA warp w takes the 32-deep K pieces
+// w, w+8, w+16, ... of the block, lane l owns column 32*b + l, and a
+// shared-memory sum over the 8 warps (in warp order) gives y.  Every lane
+// loads its weights as 16-byte vectors straight into registers (a warp reads
+// 512 contiguous bytes of the packed layout, see repack_kernel): two rounds
+// of eight loads per thread are issued before the kernel waits for the
+// previous grid, so the weight stream of this call overlaps the tail of the
+// previous one (programmatic dependent launch).
+//
+// MSD: gemv_expand_kernel runs first and writes, once per call, A_max and
+// the digits A1..A3 (section 4.1 steps 1-8, the same IEEE binary32 steps as
+// expand_kernel) as one record per (32-K piece, row): the digit bytes in the
+// order the packed weight words unpack to, so that each weight word meets
+// its digits in two dp4a per digit plane: Y_i = sum_k (w+8) * A_i -
+// 8 * sum_k A_i, exact in int32.  Per piece, (Y1/7.49 + Y2/(7.49*14.98) +
+// Y3/(7.49*14.98^2)) * A_max * scale is added to the column's fp32 sum
+// (equations 9-11: a group's pieces add up to its Y_i, and the combine is
+// linear in Y_i).
+//
+// DEQUANT: each weight word gives four exact fp16 pairs (two of them 16w)
+// and meets x through the mixed-precision fma.rn.f32.f16 (exact products,
+// fp32 sums); the group scale multiplies each piece's sum.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+#include "w4a16_kernels.cuh"
+
+namespace w4a16 {
+
+constexpr int kGemvThreads = 256;
+constexpr int kGemvWarps = kGemvThreads / 32;
+constexpr int kGemvRound = 8;                        // 16-byte loads per thread per round
+constexpr int kGemvRecWords = 28;                    // MSD record: 24 digit words, 3 sums, 1 pad
+constexpr int kGemvMaxMK = 32768;                    // M * K bound of the shared-memory operand
+
+struct GemvParams {
+    const __half* x;          // [M][K]
+    const uint8_t* w;         // packed blocks
+    const __half* scale;      // [G][N]
+    __half* y;                // [M][N]
+    const uint32_t* rec;      // MSD: [K/32][M][28] digit records
+    const float* amax;        // MSD: [M][G]
+    int M, K, N, g, G;
+    int kchunks;              // ceil(K / 128)
+    int npieces;              // K / 32
+    int nblk;                 // ceil(N / 32)
+    int ctas;                 // P
+};
+
+template <int VAR, int MR>
+struct GemvCfg {
+    static constexpr bool kIsMsd = VAR == kMsd;
+    static constexpr int kRed = kGemvWarps * MR * 32 * 4;   // cross-warp sum buffer
+    __host__ __device__ static constexpr int operand_bytes(int M, int K)
+    {
+        // MSD: the digit records and A_max; DEQUANT: x as fp16
+        return kIsMsd ? (K / 32) * M * kGemvRecWords * 4 + M * (K / 32) * 4 : M * K * 2;
+    }
+    __host__ __device__ static constexpr int smem_bytes(int M, int K)
+    {
+        return kRed + ((operand_bytes(M, K) + 15) / 16) * 16;
+    }
+};
+
+// unsigned bytes of `a` times signed bytes of `b`, summed into c
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c)
+{
+    int d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// c + a.lo * b.lo + a.hi * b.hi, fp16 inputs, products exact, fp32 adds
+__device__ __forceinline__ float fma2_f16_f32(uint32_t a2, uint32_t b2, float c)
+{
+    float d;
+    asm("{\n\t.reg .f16 al, ah, bl, bh;\n\t.reg .f32 t;\n\t"
+        "mov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.f16 t, al, bl, %3;\n\t"
+        "fma.rn.f32.f16 %0, ah, bh, t;\n\t}"
+        : "=f"(d)
+        : "r"(a2), "r"(b2), "f"(c));
+    return d;
+}
+
+// Eight packed weights -> four fp16 pairs: p0 = (w0, w1), p1 = 16 * (w2, w3),
+// p2 = (w4, w5), p3 = 16 * (w6, w7), all exact.  From the binary16 format,
+// 0x6400 | u is 1024 + u and 0x6400 | (u << 4) is 1024 + 16u; subtracting
+// 1032 and 1152 leaves w and 16w (u = w + 8).
+__device__ __forceinline__ void gemv_unpack_half(uint32_t q, uint32_t (&p)[4])
+{
+    const __half2 k1032 = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
+    const __half2 k1152 = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
+    const uint32_t q8 = q >> 8;
+    uint32_t h0 = (q & 0x000F000Fu) | 0x64006400u;
+    uint32_t h1 = (q & 0x00F000F0u) | 0x64006400u;
+    uint32_t h2 = (q8 & 0x000F000Fu) | 0x64006400u;
+    uint32_t h3 = (q8 & 0x00F000F0u) | 0x64006400u;
+    p[0] = pack_half2_bits(__hsub2(*reinterpret_cast<__half2*>(&h0), k1032));
+    p[1] = pack_half2_bits(__hsub2(*reinterpret_cast<__half2*>(&h1), k1152));
+    p[2] = pack_half2_bits(__hsub2(*reinterpret_cast<__half2*>(&h2), k1032));
+    p[3] = pack_half2_bits(__hsub2(*reinterpret_cast<__half2*>(&h3), k1152));
+}
+
+// 16 bytes of the weight stream, read once: not kept in L1
+__device__ __forceinline__ uint4 ldg_stream(const void* p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// ------------------------------------------------------------------ MSD steps 1-8 for the GEMV
+
+// One warp per (row m, span of S = max(g, 128) K values); lane l holds the
+// values 4l .. 4l+3 of each 128-value sub-chunk of the span (NSUB = S / 128
+// sub-chunks).  A_max per group (g < 128: the g/4 lanes of a group reduce
+// among themselves), then the digits in IEEE binary32 with the literal
+// operation order of steps 2-7, then per 32-K piece (8 lanes) a record of
+// 28 words: word i*8 + 2j + h holds digit plane i's bytes for the piece's
+// packed word j, low (h = 0: K offsets 8j + {0, 4, 1, 5}) or high (h = 1:
+// 8j + {2, 6, 3, 7}) nibbles -- the byte order of q & 0x0F0F0F0F and
+// (q >> 4) & 0x0F0F0F0F for a packed word q; words 24..26 hold -8 * (sum of
+// the piece's digits of plane i).  rec: [K/32][M][28]; amax: [M][G].
+template <int NSUB>
+__global__ void __launch_bounds__(256) gemv_expand_kernel(const __half* __restrict__ x, int M, int K, int g,
+                                                          uint32_t* __restrict__ rec, float* __restrict__ amax)
+{
+    // the matmul that reads the records may launch now and stream its
+    // weights; x may come from the previous kernel, and the previous matmul
+    // may still read the records this kernel overwrites
+    griddep_launch_dependents();
+    griddep_wait();
+    const int lane = threadIdx.x & 31;
+    const int span = NSUB * kKC;
+    const int nspans = (K + span - 1) / span;
+    const int G = K / g;
+    const long long wg = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) >> 5;
+    if (wg >= static_cast<long long>(M) * nspans) return;
+    const int m = static_cast<int>(wg / nspans), sp = static_cast<int>(wg % nspans);
+
+    float v[NSUB][4];
+    float am = 0.f;
+#pragma unroll
+    for (int s = 0; s < NSUB; ++s) {
+        const int k0 = sp * span + s * kKC + 4 * lane;
+        if (k0 < K) {
+            const uint2 raw = *reinterpret_cast<const uint2*>(x + static_cast<size_t>(m) * K + k0);
+            const __half2 x01 = *reinterpret_cast<const __half2*>(&raw.x);
+            const __half2 x23 = *reinterpret_cast<const __half2*>(&raw.y);
+            v[s][0] = __low2float(x01);
+            v[s][1] = __high2float(x01);
+            v[s][2] = __low2float(x23);
+            v[s][3] = __high2float(x23);
+        } else {
+            v[s][0] = v[s][1] = v[s][2] = v[s][3] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) am = fmaxf(am, fabsf(v[s][e]));
+    }
+    // A_max of each group: g >= 128 spans the warp's whole span; g < 128
+    // covers g/4 consecutive lanes
+    const int lanes_per_group = g >= kKC ? 32 : g / 4;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1)
+        if (o < lanes_per_group) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+    if ((lane % lanes_per_group) == 0) {
+        const int k0 = sp * span + 4 * lane;
+        if (k0 < K) amax[static_cast<size_t>(m) * G + k0 / g] = am;
+    }
+
+#pragma unroll
+    for (int s = 0; s < NSUB; ++s) {
+        const int k0 = sp * span + s * kKC + 4 * lane;
+        uint32_t word[3] = {0u, 0u, 0u};
+        int sum[3] = {0, 0, 0};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            int d1 = 0, d2 = 0, d3 = 0;
+            if (am != 0.f) {
+                const float t1 = __fdiv_rn(__fmul_rn(7.49f, v[s][e]), am);
+                const float a1 = rintf(t1);
+                const float t2 = __fmul_rn(__fsub_rn(t1, a1), 14.98f);
+                const float a2 = rintf(t2);
+                const float t3 = __fmul_rn(__fsub_rn(t2, a2), 14.98f);
+                const float a3 = rintf(t3);
+                d1 = static_cast<int>(a1);
+                d2 = static_cast<int>(a2);
+                d3 = static_cast<int>(a3);
+            }
+            word[0] |= (static_cast<uint32_t>(d1) & 0xFFu) << (8 * e);
+            word[1] |= (static_cast<uint32_t>(d2) & 0xFFu) << (8 * e);
+            word[2] |= (static_cast<uint32_t>(d3) & 0xFFu) << (8 * e);
+            sum[0] += d1;
+            sum[1] += d2;
+            sum[2] += d3;
+        }
+        // lanes 2j and 2j+1 of each 8-lane piece hold K offsets 8j..8j+3 and 8j+4..8j+7
+        const int pg = (sp * span + s * kKC) / 32 + (lane >> 3);
+        uint32_t* r = rec + (static_cast<size_t>(pg) * M + m) * kGemvRecWords;
+#pragma unroll
+        for (int i = 0; i < 3; ++i) {
+            const uint32_t other = __shfl_xor_sync(0xffffffffu, word[i], 1);
+            // even lane: [a0 a4 a1 a5] from (mine = a0..a3, other = a4..a7);
+            // odd lane:  [a2 a6 a3 a7] from (other = a0..a3, mine = a4..a7)
+            const uint32_t out =
+                (lane & 1) ? __byte_perm(other, word[i], 0x7362) : __byte_perm(word[i], other, 0x5140);
+            int t = sum[i];
+            t += __shfl_xor_sync(0xffffffffu, t, 1);
+            t += __shfl_xor_sync(0xffffffffu, t, 2);
+            t += __shfl_xor_sync(0xffffffffu, t, 4);
+            if (k0 < K) {   // a piece lies wholly inside or outside K (K % 32 == 0)
+                r[i * 8 + (lane & 7)] = out;
+                if ((lane & 7) == 0) r[24 + i] = static_cast<uint32_t>(-8 * t);
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ the GEMV
+
+template <int VAR, int MR>
+__global__ void __launch_bounds__(kGemvThreads, 2) gemv_kernel(const __grid_constant__ GemvParams P)
+{
+    using C = GemvCfg<VAR, MR>;
+    extern __shared__ __align__(16) uint8_t smem[];
+    float* red = reinterpret_cast<float*>(smem);                        // [8 warps][MR][32]
+    uint8_t* operand = smem + C::kRed;
+    const int rec_words = P.npieces * P.M * kGemvRecWords;
+    const uint32_t* rec_s = reinterpret_cast<const uint32_t*>(operand);
+    const float* amax_s = reinterpret_cast<const float*>(operand + rec_words * 4);
+    const __half* xs = reinterpret_cast<const __half*>(operand);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int M = P.M, K = P.K, g = P.g;
+    const int b0 = static_cast<int>((static_cast<long long>(blockIdx.x) * P.nblk) / P.ctas);
+    const int b1 = static_cast<int>((static_cast<long long>(blockIdx.x + 1) * P.nblk) / P.ctas);
+    const int ppw = (P.npieces + kGemvWarps - 1) / kGemvWarps;        // pieces per warp (upper bound)
+    const int rpb = (ppw + kGemvRound - 1) / kGemvRound;               // rounds per column block
+    const int nitems = (b1 - b0) * rpb;
+
+    // the next kernel in the stream may start its own weight stream now
+    griddep_launch_dependents();
+
+    // round i: column block b0 + i / rpb, pieces warp + 8 * (8 * (i % rpb) + j)
+    // (scales two per register: piece j's in the low / high half of sc[j / 2])
+    auto load = [&](uint4 (&buf)[kGemvRound], uint32_t (&sc)[kGemvRound / 2], int i) {
+        const int b = b0 + i / rpb, rr = i % rpb;
+        const int n = b * 32 + lane;
+        const int tile = n >> 7, r = n & 127;
+        const uint8_t* wt = P.w + static_cast<size_t>(tile) * P.kchunks * kWStage + r * 16;
+#pragma unroll
+        for (int j = 0; j < kGemvRound; ++j) {
+            const int p = warp + kGemvWarps * (kGemvRound * rr + j);
+            uint32_t h = 0u;
+            if (p < P.npieces) {
+                buf[j] = ldg_stream(wt + static_cast<size_t>(p >> 2) * kWStage + (p & 3) * 2048);
+                if (n < P.N) h = __half_as_ushort(P.scale[static_cast<size_t>((p * 32) / g) * P.N + n]);
+            }
+            if (j & 1)
+                sc[j >> 1] |= h << 16;
+            else
+                sc[j >> 1] = h;
+        }
+    };
+
+    float acc[MR];
+#pragma unroll
+    for (int m = 0; m < MR; ++m) acc[m] = 0.f;
+
+    auto compute = [&](const uint4 (&buf)[kGemvRound], const uint32_t (&sc)[kGemvRound / 2], int i) {
+        const int rr = i % rpb;
+#pragma unroll
+        for (int j = 0; j < kGemvRound; ++j) {
+            const int p = warp + kGemvWarps * (kGemvRound * rr + j);
+            if (p >= P.npieces) break;
+            const uint32_t q[4] = {buf[j].x, buf[j].y, buf[j].z, buf[j].w};
+            const float scl =
+                __half2float(__ushort_as_half(static_cast<unsigned short>(sc[j >> 1] >> (16 * (j & 1)))));
+            if constexpr (C::kIsMsd) {
+                const int grp = (p * 32) / g;
+                uint32_t lo[4], hi[4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    lo[t] = q[t] & 0x0F0F0F0Fu;
+                    hi[t] = (q[t] >> 4) & 0x0F0F0F0Fu;
+                }
+#pragma unroll
+                for (int m = 0; m < MR; ++m) {
+                    if (m >= M) break;
+                    const uint4* r4 =
+                        reinterpret_cast<const uint4*>(rec_s + (static_cast<size_t>(p) * M + m) * kGemvRecWords);
+                    const uint4 ini = r4[6];
+                    const int init[3] = {static_cast<int>(ini.x), static_cast<int>(ini.y), static_cast<int>(ini.z)};
+                    int yv[3];
+#pragma unroll
+                    for (int pl = 0; pl < 3; ++pl) {
+                        const uint4 d0 = r4[pl * 2], d1 = r4[pl * 2 + 1];
+                        int a = init[pl];
+                        a = dp4a_us(lo[0], d0.x, a);
+                        a = dp4a_us(hi[0], d0.y, a);
+                        a = dp4a_us(lo[1], d0.z, a);
+                        a = dp4a_us(hi[1], d0.w, a);
+                        a = dp4a_us(lo[2], d1.x, a);
+                        a = dp4a_us(hi[2], d1.y, a);
+                        a = dp4a_us(lo[3], d1.z, a);
+                        a = dp4a_us(hi[3], d1.w, a);
+                        yv[pl] = a;
+                    }
+                    const float v = fmaf(static_cast<float>(yv[2]), kC3,
+                                         fmaf(static_cast<float>(yv[1]), kC2, static_cast<float>(yv[0]) * kC1));
+                    acc[m] = fmaf(v, amax_s[m * P.G + grp] * scl, acc[m]);
+                }
+            } else {
+                uint32_t h[4][4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) gemv_unpack_half(q[t], h[t]);
+#pragma unroll
+                for (int m = 0; m < MR; ++m) {
+                    if (m >= M) break;
+                    const uint4* x4 = reinterpret_cast<const uint4*>(xs + static_cast<size_t>(m) * K + p * 32);
+                    float s1a = 0.f, s1b = 0.f, s16a = 0.f, s16b = 0.f;
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const uint4 xv = x4[t];             // x[8t .. 8t+7] as four pairs
+                        s1a = fma2_f16_f32(xv.x, h[t][0], s1a);
+                        s16a = fma2_f16_f32(xv.y, h[t][1], s16a);
+                        s1b = fma2_f16_f32(xv.z, h[t][2], s1b);
+                        s16b = fma2_f16_f32(xv.w, h[t][3], s16b);
+                    }
+                    const float sp = (s1a + s1b) + (s16a + s16b) * 0.0625f;
+                    acc[m] = fmaf(sp, scl, acc[m]);
+                }
+            }
+        }
+        // after the block's last round: sum the 8 warps in order, write y
+        if (rr == rpb - 1) {
+#pragma unroll
+            for (int m = 0; m < MR; ++m) red[(warp * MR + m) * 32 + lane] = acc[m];
+            __syncthreads();
+            if (tid < 32 * MR) {
+                const int m = tid >> 5, l = tid & 31;
+                const int n = (b0 + i / rpb) * 32 + l;
+                if (m < M && n < P.N) {
+                    float s = 0.f;
+#pragma unroll
+                    for (int w = 0; w < kGemvWarps; ++w) s += red[(w * MR + m) * 32 + l];
+                    P.y[static_cast<size_t>(m) * P.N + n] = __float2half_rn(s);
+                }
+            }
+            __syncthreads();
+#pragma unroll
+            for (int m = 0; m < MR; ++m) acc[m] = 0.f;
+        }
+    };
+
+    uint4 bufA[kGemvRound], bufB[kGemvRound];
+    uint32_t scA[kGemvRound / 2], scB[kGemvRound / 2];
+    if (nitems > 0) load(bufA, scA, 0);
+    if (nitems > 1) load(bufB, scB, 1);
+
+    // x and the MSD records (and whatever wrote them) are valid once the
+    // previous grid is done
+    griddep_wait();
+    if constexpr (C::kIsMsd) {
+        const uint4* src = reinterpret_cast<const uint4*>(P.rec);
+        uint4* dst = reinterpret_cast<uint4*>(operand);
+        for (int v = tid; v < rec_words / 4; v += kGemvThreads) dst[v] = src[v];
+        float* am = reinterpret_cast<float*>(operand + rec_words * 4);
+        for (int v = tid; v < M * P.G; v += kGemvThreads) am[v] = P.amax[v];
+    } else {
+        const uint4* src = reinterpret_cast<const uint4*>(P.x);
+        uint4* dst = reinterpret_cast<uint4*>(operand);
+        for (int v = tid; v < M * K / 8; v += kGemvThreads) dst[v] = src[v];
+    }
+    __syncthreads();
+
+    for (int i = 0; i < nitems; i += 2) {
+        compute(bufA, scA, i);
+        if (i + 2 < nitems) load(bufA, scA, i + 2);
+        if (i + 1 < nitems) {
+            compute(bufB, scB, i + 1);
+            if (i + 3 < nitems) load(bufB, scB, i + 3);
+        }
+    }
+}
+
+}  // namespace w4a16
