@@ -133,36 +133,6 @@ def barrier(device=None):
             dist.barrier()
 
 
-# ---------------------------------------------------------------- events inside CUDA graphs
-
-_cudart = None
-
-
-def _libcudart():
-    """The CUDA runtime torch already loaded (found in this process's maps)."""
-    global _cudart
-    if _cudart is None:
-        import ctypes
-        path = None
-        with open("/proc/self/maps") as f:
-            for line in f:
-                if "libcudart.so" in line:
-                    path = line.split()[-1]
-                    break
-        _cudart = ctypes.CDLL(path or "libcudart.so.12")
-        _cudart.cudaEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
-        _cudart.cudaEventRecordWithFlags.restype = ctypes.c_int
-    return _cudart
-
-
-def record_in_graph(event, stream):
-    """Record `event` as a timing node of the graph being captured on `stream`
-    (cudaEventRecordExternal), so it is stamped on every replay."""
-    rc = _libcudart().cudaEventRecordWithFlags(event.cuda_event, stream.cuda_stream, 1)
-    if rc != 0:
-        raise RuntimeError(f"cudaEventRecordWithFlags failed: {rc}")
-
-
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -261,15 +231,11 @@ class GpuWorkload:
         else:
             w4.w4a16_dequant_matmul(x, self.wp[k][0], self.sc[k][0], wl.M, wl.K, wl.N, wl.g, y, self.ws[op])
 
-    def step(self, s, events=None, stream=None):
+    def step(self, s):
         """One step: MSD then dequant, each on its own weight copy."""
         w4 = self.w4
         for v, op in enumerate((w4.OP_MSD, w4.OP_DEQUANT)):
-            if events is not None:
-                record_in_graph(events[v][0], stream)
             self.call(op, 2 * s + v)
-            if events is not None:
-                record_in_graph(events[v][1], stream)
 
 
 def launches_per_step(grouped):
@@ -304,25 +270,16 @@ def run_gpu(args, wl, rank, world, local):
     period = max(1, G.copies // 2)
     per_graph = period * max(1, 400 // period)
     nrep, rem = divmod(args.steps, per_graph)
-    events = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(period)] for _ in range(2)]
-    for pair in events:
-        for a, b in pair:          # materialise the CUDA events before capture
-            a.record(stream)
-            b.record(stream)
-    stream.synchronize()
-
-    def capture(n, with_events):
+    def capture(n, body):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.stream(stream):
             with torch.cuda.graph(g, stream=stream):
                 for s in range(n):
-                    ev = [events[0][s], events[1][s]] if (with_events and s < period) else None
-                    G.step(s, ev, stream)
+                    body(s)
         return g
 
-    graph = capture(per_graph, True) if nrep else None
-    tail = capture(rem, False) if rem else None
+    graph = capture(per_graph, G.step) if nrep else None
+    tail = capture(rem, G.step) if rem else None
     # untimed replay to warm the graph
     with torch.cuda.stream(stream):
         if graph is not None:
@@ -355,12 +312,22 @@ def run_gpu(args, wl, rank, world, local):
         if w4.w4a16_read_status(G.ws[op], stream) != 0:
             raise RuntimeError("device wait timed out during the timed region")
 
-    # per-call durations (events around each call in the last graph replay)
+    # per-call durations of each variant in steady state: a graph of
+    # consecutive calls of that variant alone (weights still rotating),
+    # replayed once untimed and once between two events on the launch stream
     per_call_us = {}
-    if graph is not None:
-        for v, name in enumerate(("msd", "dequant")):
-            d = [events[v][s][0].elapsed_time(events[v][s][1]) * 1e3 for s in range(period)]
-            per_call_us[name] = float(np.mean(d))
+    n_op = 2 * period * max(1, 100 // period)
+    for op, name in ((w4.OP_MSD, "msd"), (w4.OP_DEQUANT, "dequant")):
+        g_op = capture(n_op, lambda s, op=op: G.call(op, s))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            g_op.replay()
+            e0.record(stream)
+            g_op.replay()
+            e1.record(stream)
+        stream.synchronize()
+        per_call_us[name] = e0.elapsed_time(e1) * 1e3 / n_op
+        del g_op
 
     # end to end through the public API with host buffers: per step, the
     # activations go host->device from pinned memory, both variants run, and
@@ -407,7 +374,8 @@ def run_gpu(args, wl, rank, world, local):
         "config": {"workload": f"{wl.name}: M={wl.M} K={wl.K} N={wl.N} g={wl.g}" + (f" E={wl.E}" if wl.E > 1 else "")
                    + "; one step = MSD matmul + dequant matmul",
                    "l2": f"weights rotated over {G.copies} copies (> L2) between calls",
-                   "timing": f"CUDA graph of {per_graph} steps replayed; events on the launch stream",
+                   "timing": f"CUDA graph of {per_graph} steps replayed; events on the launch stream; per-call times from "
+                             f"graphs of {n_op} calls of one variant",
                    "parallelism": f"{world} independent replica(s), one per GPU" if world > 1 else "single GPU",
                    "tflops_per_s": round(flops_step * args.steps * world / (ms * 1e-3) / 1e12, 3)},
         "roofline": roof, "detail": detail, "e2e": e2e,

@@ -10,9 +10,11 @@
 //
 // Work split: output columns only.  The columns form blocks of 32 (one warp
 // width); CTA c of P takes blocks [c*B/P, (c+1)*B/P) and all of K, so no
-// partial sums leave the CTA.  Inside a CTA warp w takes the 32-deep K pieces
-// w, w+8, w+16, ... of the block, lane l owns column 32*b + l, and a
-// shared-memory sum over the 8 warps (in warp order) gives y.  Every lane
+// partial sums leave the CTA.  Inside a CTA warp w takes a contiguous run of
+// whole groups (G/8 of them) of the block, lane l owns column 32*b + l, and
+// a shared-memory sum over the 8 warps (in warp order) gives y.  Sums stay
+// per group (integer Y_i for MSD) until the group's last piece, where the
+// scale (and A_max) is applied once.  Every lane
 // loads its weights as 16-byte vectors straight into registers (a warp reads
 // 512 contiguous bytes of the packed layout, see repack_kernel): two rounds
 // of eight loads per thread are issued before the kernel waits for the
@@ -29,9 +31,11 @@
 // (equations 9-11: a group's pieces add up to its Y_i, and the combine is
 // linear in Y_i).
 //
-// DEQUANT: each weight word gives four exact fp16 pairs (two of them 16w)
-// and meets x through the mixed-precision fma.rn.f32.f16 (exact products,
-// fp32 sums); the group scale multiplies each piece's sum.
+// DEQUANT: each weight word gives four fp16 pairs of biased values (1024 + u
+// or 1024 + 16u, exact) that meet x through the mixed-precision
+// fma.rn.f32.f16 (exact products, fp32 sums); one correction per piece made
+// from the sums of x removes the biases, and the group scale multiplies
+// each piece's sum.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -69,8 +73,9 @@ struct GemvCfg {
     static constexpr int kRed = kGemvWarps * MR * 32 * 4;   // cross-warp sum buffer
     __host__ __device__ static constexpr int operand_bytes(int M, int K)
     {
-        // MSD: the digit records and A_max; DEQUANT: x as fp16
-        return kIsMsd ? (K / 32) * M * kGemvRecWords * 4 + M * (K / 32) * 4 : M * K * 2;
+        // MSD: the digit records and A_max; DEQUANT: x as fp16 and one fp32
+        // bias correction per (32-K piece, row)
+        return kIsMsd ? (K / 32) * M * kGemvRecWords * 4 + M * (K / 32) * 4 : M * K * 2 + (K / 32) * M * 4;
     }
     __host__ __device__ static constexpr int smem_bytes(int M, int K)
     {
@@ -99,23 +104,18 @@ __device__ __forceinline__ float fma2_f16_f32(uint32_t a2, uint32_t b2, float c)
     return d;
 }
 
-// Eight packed weights -> four fp16 pairs: p0 = (w0, w1), p1 = 16 * (w2, w3),
-// p2 = (w4, w5), p3 = 16 * (w6, w7), all exact.  From the binary16 format,
-// 0x6400 | u is 1024 + u and 0x6400 | (u << 4) is 1024 + 16u; subtracting
-// 1032 and 1152 leaves w and 16w (u = w + 8).
-__device__ __forceinline__ void gemv_unpack_half(uint32_t q, uint32_t (&p)[4])
+// Eight packed weights -> four fp16 pairs holding biased values, exactly:
+// from the binary16 format, 0x6400 | u is 1024 + u and 0x6400 | (u << 4) is
+// 1024 + 16u (u = w + 8), so p0 = 1024 + (u0, u1), p1 = 1024 + 16 (u2, u3),
+// p2 = 1024 + (u4, u5), p3 = 1024 + 16 (u6, u7).  The biases are removed once
+// per piece (see gemv_kernel), not per weight.
+__device__ __forceinline__ void gemv_unpack_biased(uint32_t q, uint32_t (&p)[4])
 {
-    const __half2 k1032 = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
-    const __half2 k1152 = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
     const uint32_t q8 = q >> 8;
-    uint32_t h0 = (q & 0x000F000Fu) | 0x64006400u;
-    uint32_t h1 = (q & 0x00F000F0u) | 0x64006400u;
-    uint32_t h2 = (q8 & 0x000F000Fu) | 0x64006400u;
-    uint32_t h3 = (q8 & 0x00F000F0u) | 0x64006400u;
-    p[0] = pack_half2_bits(__hsub2(*reinterpret_cast<__half2*>(&h0), k1032));
-    p[1] = pack_half2_bits(__hsub2(*reinterpret_cast<__half2*>(&h1), k1152));
-    p[2] = pack_half2_bits(__hsub2(*reinterpret_cast<__half2*>(&h2), k1032));
-    p[3] = pack_half2_bits(__hsub2(*reinterpret_cast<__half2*>(&h3), k1152));
+    p[0] = (q & 0x000F000Fu) | 0x64006400u;
+    p[1] = (q & 0x00F000F0u) | 0x64006400u;
+    p[2] = (q8 & 0x000F000Fu) | 0x64006400u;
+    p[3] = (q8 & 0x00F000F0u) | 0x64006400u;
 }
 
 // 16 bytes of the weight stream, read once: not kept in L1
@@ -248,32 +248,46 @@ __global__ void __launch_bounds__(kGemvThreads, 2) gemv_kernel(const __grid_cons
     const uint32_t* rec_s = reinterpret_cast<const uint32_t*>(operand);
     const float* amax_s = reinterpret_cast<const float*>(operand + rec_words * 4);
     const __half* xs = reinterpret_cast<const __half*>(operand);
+    float* xcorr = reinterpret_cast<float*>(operand + P.M * P.K * 2);   // DEQUANT: [K/32][M]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int M = P.M, K = P.K, g = P.g;
+    const int M = P.M, K = P.K;
     const int b0 = static_cast<int>((static_cast<long long>(blockIdx.x) * P.nblk) / P.ctas);
     const int b1 = static_cast<int>((static_cast<long long>(blockIdx.x + 1) * P.nblk) / P.ctas);
-    const int ppw = (P.npieces + kGemvWarps - 1) / kGemvWarps;        // pieces per warp (upper bound)
-    const int rpb = (ppw + kGemvRound - 1) / kGemvRound;               // rounds per column block
+    // warp w takes the whole groups [w*G/8, (w+1)*G/8), i.e. a contiguous run
+    // of 32-K pieces [pw0, pw1); a group is ppg pieces
+    const int ppg = P.g / 32;
+    const int pw0 = ((warp * P.G) / kGemvWarps) * ppg;
+    const int pw1 = (((warp + 1) * P.G) / kGemvWarps) * ppg;
+    // rounds per column block: the same for every warp (the block-end sum
+    // below is a CTA-wide barrier), sized for the warp with the most groups
+    const int rpb = (((P.G + kGemvWarps - 1) / kGemvWarps) * ppg + kGemvRound - 1) / kGemvRound;
     const int nitems = (b1 - b0) * rpb;
 
     // the next kernel in the stream may start its own weight stream now
     griddep_launch_dependents();
 
-    // round i: column block b0 + i / rpb, pieces warp + 8 * (8 * (i % rpb) + j)
-    // (scales two per register: piece j's in the low / high half of sc[j / 2])
+    // round i: column block b0 + i / rpb, pieces pw0 + 8 * (i % rpb) + j; the
+    // scale of a group is loaded with its last piece (two per register: piece
+    // j's in the low / high half of sc[j / 2])
     auto load = [&](uint4 (&buf)[kGemvRound], uint32_t (&sc)[kGemvRound / 2], int i) {
         const int b = b0 + i / rpb, rr = i % rpb;
         const int n = b * 32 + lane;
         const int tile = n >> 7, r = n & 127;
         const uint8_t* wt = P.w + static_cast<size_t>(tile) * P.kchunks * kWStage + r * 16;
+        const int pbase = pw0 + kGemvRound * rr;
+        int grp = pbase / ppg, pos = (kGemvRound * rr) % ppg;   // group of the next piece, pieces done in it
 #pragma unroll
         for (int j = 0; j < kGemvRound; ++j) {
-            const int p = warp + kGemvWarps * (kGemvRound * rr + j);
+            const int p = pbase + j;
             uint32_t h = 0u;
-            if (p < P.npieces) {
+            if (p < pw1) {
                 buf[j] = ldg_stream(wt + static_cast<size_t>(p >> 2) * kWStage + (p & 3) * 2048);
-                if (n < P.N) h = __half_as_ushort(P.scale[static_cast<size_t>((p * 32) / g) * P.N + n]);
+                if (++pos == ppg) {
+                    if (n < P.N) h = __half_as_ushort(P.scale[static_cast<size_t>(grp) * P.N + n]);
+                    ++grp;
+                    pos = 0;
+                }
             }
             if (j & 1)
                 sc[j >> 1] |= h << 16;
@@ -283,20 +297,26 @@ __global__ void __launch_bounds__(kGemvThreads, 2) gemv_kernel(const __grid_cons
     };
 
     float acc[MR];
+    int yacc[MR][3];       // MSD: the group's Y1..Y3 so far
+    float gsum[MR];        // DEQUANT: the group's sum_k x w so far
 #pragma unroll
-    for (int m = 0; m < MR; ++m) acc[m] = 0.f;
+    for (int m = 0; m < MR; ++m) {
+        acc[m] = 0.f;
+        gsum[m] = 0.f;
+        yacc[m][0] = yacc[m][1] = yacc[m][2] = 0;
+    }
 
     auto compute = [&](const uint4 (&buf)[kGemvRound], const uint32_t (&sc)[kGemvRound / 2], int i) {
         const int rr = i % rpb;
+        const int pbase = pw0 + kGemvRound * rr;
+        int grp = pbase / ppg, pos = (kGemvRound * rr) % ppg;
 #pragma unroll
         for (int j = 0; j < kGemvRound; ++j) {
-            const int p = warp + kGemvWarps * (kGemvRound * rr + j);
-            if (p >= P.npieces) break;
+            const int p = pbase + j;
+            if (p >= pw1) break;
             const uint32_t q[4] = {buf[j].x, buf[j].y, buf[j].z, buf[j].w};
-            const float scl =
-                __half2float(__ushort_as_half(static_cast<unsigned short>(sc[j >> 1] >> (16 * (j & 1)))));
+            const bool group_end = ++pos == ppg;
             if constexpr (C::kIsMsd) {
-                const int grp = (p * 32) / g;
                 uint32_t lo[4], hi[4];
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
@@ -310,11 +330,10 @@ __global__ void __launch_bounds__(kGemvThreads, 2) gemv_kernel(const __grid_cons
                         reinterpret_cast<const uint4*>(rec_s + (static_cast<size_t>(p) * M + m) * kGemvRecWords);
                     const uint4 ini = r4[6];
                     const int init[3] = {static_cast<int>(ini.x), static_cast<int>(ini.y), static_cast<int>(ini.z)};
-                    int yv[3];
 #pragma unroll
                     for (int pl = 0; pl < 3; ++pl) {
                         const uint4 d0 = r4[pl * 2], d1 = r4[pl * 2 + 1];
-                        int a = init[pl];
+                        int a = yacc[m][pl] + init[pl];
                         a = dp4a_us(lo[0], d0.x, a);
                         a = dp4a_us(hi[0], d0.y, a);
                         a = dp4a_us(lo[1], d0.z, a);
@@ -323,16 +342,32 @@ __global__ void __launch_bounds__(kGemvThreads, 2) gemv_kernel(const __grid_cons
                         a = dp4a_us(hi[2], d1.y, a);
                         a = dp4a_us(lo[3], d1.z, a);
                         a = dp4a_us(hi[3], d1.w, a);
-                        yv[pl] = a;
+                        yacc[m][pl] = a;
                     }
-                    const float v = fmaf(static_cast<float>(yv[2]), kC3,
-                                         fmaf(static_cast<float>(yv[1]), kC2, static_cast<float>(yv[0]) * kC1));
-                    acc[m] = fmaf(v, amax_s[m * P.G + grp] * scl, acc[m]);
+                }
+                if (group_end) {
+                    const float scl =
+                        __half2float(__ushort_as_half(static_cast<unsigned short>(sc[j >> 1] >> (16 * (j & 1)))));
+#pragma unroll
+                    for (int m = 0; m < MR; ++m) {
+                        if (m >= M) break;
+                        const float v = fmaf(static_cast<float>(yacc[m][2]), kC3,
+                                             fmaf(static_cast<float>(yacc[m][1]), kC2,
+                                                  static_cast<float>(yacc[m][0]) * kC1));
+                        acc[m] = fmaf(v, amax_s[m * P.G + grp] * scl, acc[m]);
+                        yacc[m][0] = yacc[m][1] = yacc[m][2] = 0;
+                    }
+                    ++grp;
+                    pos = 0;
                 }
             } else {
+                // with A = K offsets {0,1,4,5} and B = {2,3,6,7} of each word,
+                // s1 = sum_A x (1024 + u) and s16 = sum_B x (1024 + 16u), so the
+                // piece's sum_k x w = s1 + s16 / 16 - 1032 X_A - 72 X_B, the
+                // last two terms (sums of x alone) precomputed per piece
                 uint32_t h[4][4];
 #pragma unroll
-                for (int t = 0; t < 4; ++t) gemv_unpack_half(q[t], h[t]);
+                for (int t = 0; t < 4; ++t) gemv_unpack_biased(q[t], h[t]);
 #pragma unroll
                 for (int m = 0; m < MR; ++m) {
                     if (m >= M) break;
@@ -346,8 +381,17 @@ __global__ void __launch_bounds__(kGemvThreads, 2) gemv_kernel(const __grid_cons
                         s1b = fma2_f16_f32(xv.z, h[t][2], s1b);
                         s16b = fma2_f16_f32(xv.w, h[t][3], s16b);
                     }
-                    const float sp = (s1a + s1b) + (s16a + s16b) * 0.0625f;
-                    acc[m] = fmaf(sp, scl, acc[m]);
+                    gsum[m] += (s1a + s1b) + fmaf(s16a + s16b, 0.0625f, xcorr[p * M + m]);
+                }
+                if (group_end) {
+                    const float scl =
+                        __half2float(__ushort_as_half(static_cast<unsigned short>(sc[j >> 1] >> (16 * (j & 1)))));
+#pragma unroll
+                    for (int m = 0; m < MR; ++m) {
+                        acc[m] = fmaf(gsum[m], scl, acc[m]);
+                        gsum[m] = 0.f;
+                    }
+                    pos = 0;
                 }
             }
         }
@@ -390,6 +434,25 @@ __global__ void __launch_bounds__(kGemvThreads, 2) gemv_kernel(const __grid_cons
         const uint4* src = reinterpret_cast<const uint4*>(P.x);
         uint4* dst = reinterpret_cast<uint4*>(operand);
         for (int v = tid; v < M * K / 8; v += kGemvThreads) dst[v] = src[v];
+        __syncthreads();
+        // per (piece, row): -(1032 X_A + 72 X_B), X_A / X_B the sums of x over
+        // the offsets {0,1,4,5} / {2,3,6,7} of each 8-value word
+        for (int v = tid; v < P.npieces * M; v += kGemvThreads) {
+            const int pc = v / M, m = v % M;
+            const uint4* x4 = reinterpret_cast<const uint4*>(xs + static_cast<size_t>(m) * K + pc * 32);
+            float xa = 0.f, xb = 0.f;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const uint4 xv = x4[t];
+                const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&xv.x));
+                const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&xv.y));
+                const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&xv.z));
+                const float2 f3 = __half22float2(*reinterpret_cast<const __half2*>(&xv.w));
+                xa += (f0.x + f0.y) + (f2.x + f2.y);
+                xb += (f1.x + f1.y) + (f3.x + f3.y);
+            }
+            xcorr[v] = -fmaf(1032.f, xa, 72.f * xb);
+        }
     }
     __syncthreads();
 
