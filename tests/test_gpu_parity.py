@@ -148,7 +148,7 @@ def test_dequant_small(cuda_lib, M, K, N, g):
 
 
 @pytest.mark.parametrize("M,K,N,g", [(16, 256, 256, 64), (5, 384, 136, 64), (3, 512, 256, 256),
-                                     (9, 512, 384, 32), (70, 512, 256, 64)])
+                                     (9, 512, 384, 32), (70, 512, 256, 64), (6, 768, 264, 384)])
 def test_msd_yint_bit_exact(cuda_lib, M, K, N, g):
     w4 = cuda_lib
     c = make_case(M, K, N, g, seed=99 + M + g)
@@ -229,6 +229,35 @@ def test_gemv_dequant(cuda_lib, M, K, N, g):
     dev = upload(w4, c)
     y = run_dense(w4, w4.OP_DEQUANT, c, dev)
     assert_deq_close(y, oracle.dequant(c.x, c.wp[0], c.scale[0], g), f"gemv dequant {M}x{K}x{N} g{g}")
+
+
+# Decode-sized shapes for both variants (the CUDA-core GEMV at M <= 4, the
+# tensor-core decode tile above): every group size including 384 (groups
+# that cut 128-deep chunks), ragged N, K not a multiple of 1024 or of 128,
+# one and several column blocks per CTA.
+DECODE = [
+    # (M, K, N, g)                       what it covers
+    (7, 1536, 264, 64),                  # odd M, partial stage, ragged N
+    (12, 3072, 520, 384),                # group of 384 (stages cut groups), 3 stages
+    (4, 1152, 776, 384),                 # MSD with 3 sub-chunks per span, partial last stage
+    (3, 8192, 96, 512),                  # 8 stages, one tile, N = 3 blocks
+    (1, 640, 4104, 32),                  # 129 column blocks over the SMs, ragged last block
+    (2, 160, 520, 32),                   # K of 5 pieces (not a multiple of 128)
+    (16, 1024, 2048, 128),               # the full 16 MMA rows, exactly one stage
+    (5, 2048, 18432, 64),                # several column blocks per CTA
+]
+
+
+@pytest.mark.parametrize("M,K,N,g", DECODE)
+def test_decode_shapes_both_variants(cuda_lib, M, K, N, g):
+    w4 = cuda_lib
+    c = make_case(M, K, N, g, seed=M * 1009 + K * 13 + N * 7 + g)
+    c.x[M - 1, g:2 * g] = 0              # an all-zero group
+    dev = upload(w4, c)
+    assert_msd_close(run_dense(w4, w4.OP_MSD, c, dev), oracle.msd(c.x, c.wp[0], c.scale[0], g),
+                     f"decode msd {M}x{K}x{N} g{g}")
+    assert_deq_close(run_dense(w4, w4.OP_DEQUANT, c, dev), oracle.dequant(c.x, c.wp[0], c.scale[0], g),
+                     f"decode dequant {M}x{K}x{N} g{g}")
 
 
 def test_gemv_repeat_calls_are_deterministic(cuda_lib):

@@ -323,6 +323,7 @@ w4a16_status launch_expand(const void* x, int M, int K, int g, int8_t* xq, float
         case 2: e = launch_expand_vpl<2>(blocks, xh, M, K, g, xq, amax, s); break;
         case 4: e = launch_expand_vpl<4>(blocks, xh, M, K, g, xq, amax, s); break;
         case 8: e = launch_expand_vpl<8>(blocks, xh, M, K, g, xq, amax, s); break;
+        case 12: e = launch_expand_vpl<12>(blocks, xh, M, K, g, xq, amax, s); break;
         case 16: e = launch_expand_vpl<16>(blocks, xh, M, K, g, xq, amax, s); break;
         default: return W4A16_ERR_UNSUPPORTED;
     }
