@@ -287,13 +287,13 @@ w4a16_status launch_for(int op, int TT, const CUtensorMap& map, const GemmParams
         // the Y_int debug window is a separate instance, off the hot kernels
         if (P.dbg_yint != nullptr) {
             if (TT == 16) return launch_gemm<kMsd, 16, 8, 12, 2, 1, 4, false, true>(map, P, grid, s);
-            return launch_gemm<kMsd, 64, 4, 4, 1, 2, 1, false, true>(map, P, grid, s);
+            return launch_gemm<kMsd, 64, 4, 4, 2, 2, 1, false, true>(map, P, grid, s);
         }
-        if (TT == 16) return launch_gemm<kMsd, 16, 8, 12, 2, 1, 4, false>(map, P, grid, s);
-        return launch_gemm<kMsd, 64, 4, 4, 1, 2, 1, false>(map, P, grid, s);
+        if (TT == 16) return launch_gemm<kMsd, 16, 8, 12, 2, 2, 4, false>(map, P, grid, s);
+        return launch_gemm<kMsd, 64, 4, 4, 2, 2, 1, false>(map, P, grid, s);
     }
-    if (TT == 16) return launch_gemm<kDeq, 16, 4, 12, 2, 1, 4, true>(map, P, grid, s);
-    return launch_gemm<kDeq, 128, 4, 4, 1, 1, 1, false>(map, P, grid, s);
+    if (TT == 16) return launch_gemm<kDeq, 16, 4, 12, 2, 2, 4, true>(map, P, grid, s);
+    return launch_gemm<kDeq, 128, 4, 4, 2, 1, 1, false>(map, P, grid, s);
 }
 
 template <int VPL>

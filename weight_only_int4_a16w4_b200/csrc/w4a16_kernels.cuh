@@ -146,10 +146,17 @@ struct GemmCfg {
     static constexpr int kWarps = kCtrlWarps + 4 * NCONV + 4 * NEPI;
     static constexpr int kThreads = 32 * kWarps;
     static constexpr int kEpiThreads = 128 * NEPI;
-    static constexpr int kTokPerEpi = TT / NEPI;
+    // decode tile with several epilogue groups: group eg takes the K groups
+    // j = eg, eg + NEPI, ... for all TT tokens (the per-group work is short
+    // and latency-bound, so groups in flight overlap); otherwise the groups
+    // split the tokens
+    static constexpr bool kEpiRR = TT == 16 && NEPI > 1;
+    static constexpr int kTokPerEpi = kEpiRR ? TT : TT / NEPI;
     static constexpr int kRedBytes = TT == 16 ? TT * kBN * 4 + 256 : 0;     // split-K partials (decode tile only)
+    static constexpr int kRRBytes = kEpiRR ? (NEPI - 1) * TT * kBN * 4 : 0; // partial sums of groups 1..NEPI-1
     static constexpr int kNumBars = 3 * ST + 2 * WST + 2 * kNBuf + kMaxIssuers;
-    static constexpr int kSmem = ST * kStage + WST * kWSlot + kRedBytes + 1024 + 8 * kNumBars + 16 + 2 * TT * 4 + 16;
+    static constexpr int kSmem = ST * kStage + WST * kWSlot + kRedBytes + kRRBytes + 1024 + 8 * kNumBars + 16 +
+                                 2 * TT * 4 * NEPI + 16;
     static_assert(kColsUsed <= 512, "Tensor Memory overflow");
     static_assert(kMmaN % 16 == 0 && kMmaN >= 16 && kMmaN <= 256, "MMA N out of range");
     static_assert(TT % 16 == 0 && kTokPerEpi % 16 == 0, "token tile must split into 16-token pieces");
@@ -158,6 +165,7 @@ struct GemmCfg {
     static_assert(ST % NCONV == 0 && ST % NISS == 0 && WST % NCONV == 0, "stages must split evenly over the groups");
     static_assert(NISS == 1 || NISS == 2 || NISS == 4, "1, 2 or 4 MMA issuers");
     static_assert(!SEPI || !kIsMsd, "SEPI is a DEQUANT option");
+    static_assert(!kEpiRR || (kGroupAcc && kNBuf % NEPI == 0), "round-robin epilogue needs per-group buffers");
 };
 
 // ------------------------------------------------------------------ helpers
@@ -352,10 +360,10 @@ __device__ __forceinline__ bool resolve_tile(const GemmParams& P, int TT, TileCo
     return false;
 }
 
-// MSD accumulators start every group at this bias: an int32 accumulator
-// holding 0x4B400000 + Y reads, as a binary32, exactly 12582912 + Y for
-// |Y| < 2^22 (1.5 * 2^23 has a unit last place), so the epilogue turns Y into
-// a float with one exact subtraction instead of an int -> float conversion.
+// int32 -> binary32 for the MSD accumulators: 0x4B400000 + Y, read as a
+// binary32, is exactly 12582912 + Y for |Y| < 2^22 (1.5 * 2^23 has a unit
+// last place), so one integer add and one exact subtraction convert Y
+// (|Y| <= 7 * 8 * g <= 28672) without the slower int -> float unit.
 constexpr uint32_t kAccBiasBits = 0x4B400000u;
 constexpr float kAccBias = 12582912.0f;
 // Equation 10 with 1/7.49 factored out: Y1 + Y2/14.98 + Y3/14.98^2.
@@ -371,7 +379,8 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* wsm = smem + ST * C::kStage;                              // weight slots
     float* red = reinterpret_cast<float*>(wsm + WST * C::kWSlot);      // split-K partials pushed by the cluster
-    uint64_t* bars = reinterpret_cast<uint64_t*>(wsm + WST * C::kWSlot + C::kRedBytes);
+    float* rr_part = reinterpret_cast<float*>(wsm + WST * C::kWSlot + C::kRedBytes);   // [NEPI-1][TT][128]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(wsm + WST * C::kWSlot + C::kRedBytes + C::kRRBytes);
     uint64_t* bfull_bar = bars;                 // [ST] activation tile landed
     uint64_t* sfree_bar = bfull_bar + ST;       // [ST] operand stage free again (MMA done)
     uint64_t* afull_bar = sfree_bar + ST;       // [ST] A operand written to Tensor Memory
@@ -382,8 +391,8 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
     uint64_t* done_bar = accempty_bar + C::kNBuf;    // [kMaxIssuers] all MMAs of an issuer completed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + C::kMaxIssuers);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    // [2][TT] floats read as float4: round up to a 16-byte boundary (the
-    // barriers before it end on an 8-byte boundary only)
+    // [NEPI][2][TT] floats read as float4: round up to a 16-byte boundary
+    // (the barriers before it end on an 8-byte boundary only)
     float* amax_sm = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(tmem_slot + 4) + 15) & ~uintptr_t(15));
 
     TileCoord tc;
@@ -414,7 +423,7 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
         }
         for (int b = 0; b < C::kNBuf; ++b) {
             mbar_init(smem_addr(&accfull_bar[b]), 1);
-            mbar_init(smem_addr(&accempty_bar[b]), 4 * NEPI);
+            mbar_init(smem_addr(&accempty_bar[b]), C::kEpiRR ? 4 : 4 * NEPI);
         }
         for (int q = 0; q < C::kMaxIssuers; ++q) mbar_init(smem_addr(&done_bar[q]), 1);
         *abort_flag = 0;
@@ -537,9 +546,9 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
                         const int st_ = step0 + j;
                         const int grel = gpow2 ? (st_ >> gshift) : (st_ / gsteps);     // group within the split
                         const int gpos = st_ - grel * gsteps;                          // step within the group
-                        const int ab = (grp0 + grel) % C::kNBuf;
+                        const int ab = grel % C::kNBuf;
                         if (gpos == 0) {
-                            // the epilogue has read this buffer (MSD: and reset it to the bias)
+                            // the epilogue has read this buffer
                             if (!mbar_wait(smem_addr(&accempty_bar[ab]), (grel / C::kNBuf) & 1, tmo, P.status,
                                            abort_flag)) {
                                 failed = true;
@@ -550,7 +559,8 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
                         }
                         const uint32_t d = tmem + ab * C::kAccStride;
                         if (lane == 0) {
-                            if (C::kIsMsd) mma_i8_ts(d, a_base + 8 * j, bd, idesc, 1u);
+                            // a group's first K step overwrites the buffer
+                            if (C::kIsMsd) mma_i8_ts(d, a_base + 8 * j, bd, idesc, gpos == 0 ? 0u : 1u);
                             else mma_f16_ts(d, a_base + 8 * j, bd, idesc, gpos == 0 ? 0u : 1u);
                             if (i == 2 && j < 4) W4A16_TRACE_AT(60 + j);
                             if (gpos == gsteps - 1) tc_commit(smem_addr(&accfull_bar[ab]));
@@ -654,15 +664,16 @@ W4A16_ROLE_UNROLL
         }
     } else if (warp >= C::kEpiWarp0) {
         // ============================ epilogue ============================
-        const int eg = (warp - C::kEpiWarp0) >> 2;             // epilogue group: a slice of the tokens
-        const int et = threadIdx.x - 32 * C::kEpiWarp0;        // 0 .. kEpiThreads-1
+        const int eg = (warp - C::kEpiWarp0) >> 2;             // epilogue group
+        // thread index within the threads that share the A_max ring
+        const int et = threadIdx.x - 32 * (C::kEpiRR ? C::kEpiWarp0 + 4 * eg : C::kEpiWarp0);
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32);
         const int r = lane_base + lane;
         const int n = n0 + r;
         const bool n_ok = n < P.N;
         const int nt = tc.t_end - tc.t0;
         constexpr int TE = C::kTokPerEpi;
-        const int tb = eg * TE;                                 // first token of this group
+        const int tb = C::kEpiRR ? 0 : eg * TE;                 // first token of this group
         const uint32_t t_addr = tmem + (lane_base << 16);
         float acc[TE];
 #pragma unroll
@@ -670,44 +681,35 @@ W4A16_ROLE_UNROLL
         bool ok = true;
 
         if (C::kGroupAcc) {
-            if (C::kIsMsd) {
-                // every accumulator buffer starts at the bias
-#pragma unroll
-                for (int b = 0; b < C::kNBuf; ++b)
-#pragma unroll
-                    for (int rr = 0; rr < 3; ++rr)
-#pragma unroll
-                        for (int c = 0; c < TE / 8; ++c)
-                            tmem_st8_fill(t_addr + b * C::kAccStride + rr * TT + tb + 8 * c, kAccBiasBits);
-                tmem_st_wait();
-                tc_fence_before();
-            }
             __syncwarp();
-            if (lane == 0)          // release every buffer to the MMA
-                for (int b = 0; b < C::kNBuf; ++b) mbar_arrive(smem_addr(&accempty_bar[b]));
+            if (lane == 0)          // release every buffer (this group's, round-robin) to the MMA
+                for (int b = 0; b < C::kNBuf; ++b)
+                    if (!C::kEpiRR || b % NEPI == eg) mbar_arrive(smem_addr(&accempty_bar[b]));
             griddep_wait();    // A_max comes from the expansion kernel; y is shared with earlier kernels
             if (warp == C::kEpiWarp0 && lane == 0) W4A16_TRACE_AT(52);
 
             const int ngroups = min(kc1 * kKC, P.K) / P.g - grp0;
             const __half* sc_e = P.scale[tc.e];
+            const int jstep = C::kEpiRR ? NEPI : 1, j0 = C::kEpiRR ? eg : 0;
             float am_next = 0.f, sc_next = 0.f;
-            if (ngroups > 0) {
-                if (C::kIsMsd && et < nt) am_next = __ldg(P.amax + static_cast<size_t>(grp0) * P.M + tc.t0 + et);
-                if (n_ok && sc_e) sc_next = __half2float(sc_e[static_cast<size_t>(grp0) * P.N + n]);
+            if (j0 < ngroups) {
+                if (C::kIsMsd && et < nt) am_next = __ldg(P.amax + static_cast<size_t>(grp0 + j0) * P.M + tc.t0 + et);
+                if (n_ok && sc_e) sc_next = __half2float(sc_e[static_cast<size_t>(grp0 + j0) * P.N + n]);
             }
-            for (int j = 0; j < ngroups; ++j) {
+            for (int j = j0, jj = 0; j < ngroups; j += jstep, ++jj) {
                 const int grp = grp0 + j;
-                const int ab = grp % C::kNBuf;
+                const int ab = j % C::kNBuf;
                 const uint32_t abph = (j / C::kNBuf) & 1;
-                float* am_slot = amax_sm + (j & 1) * TT;
+                float* am_slot = amax_sm + ((C::kEpiRR ? eg : 0) * 2 + (jj & 1)) * TT;
                 if (C::kIsMsd && et < TT) am_slot[et] = am_next;
                 const float sc = sc_next;
-                if (j + 1 < ngroups) {           // prefetch the next group's A_max and scale
+                if (j + jstep < ngroups) {       // prefetch the next group's A_max and scale
                     if (C::kIsMsd)
-                        am_next = (et < nt) ? __ldg(P.amax + static_cast<size_t>(grp + 1) * P.M + tc.t0 + et) : 0.f;
-                    if (n_ok && sc_e) sc_next = __half2float(sc_e[static_cast<size_t>(grp + 1) * P.N + n]);
+                        am_next = (et < nt) ? __ldg(P.amax + static_cast<size_t>(grp + jstep) * P.M + tc.t0 + et) : 0.f;
+                    if (n_ok && sc_e) sc_next = __half2float(sc_e[static_cast<size_t>(grp + jstep) * P.N + n]);
                 }
-                if (C::kIsMsd) named_bar_sync(1, C::kEpiThreads);   // every epilogue thread, every group
+                // every thread that shares the A_max ring, every group
+                if (C::kIsMsd) named_bar_sync(1 + (C::kEpiRR ? eg : 0), C::kEpiRR ? 128 : C::kEpiThreads);
                 if (ok && !mbar_wait(smem_addr(&accfull_bar[ab]), abph, tmo, P.status, abort_flag)) ok = false;
                 if (!ok) continue;
                 if (warp == C::kEpiWarp0 && lane == 0 && j < 8) W4A16_TRACE_AT(36 + j);
@@ -727,10 +729,12 @@ W4A16_ROLE_UNROLL
                         tmem_ld_wait();
 #pragma unroll
                         for (int qq = 0; qq < 8; ++qq) {
-                            // exact Y_i as floats, then equation 10 and equation 11's running sum
-                            const float d1 = __uint_as_float(y1[qq]) - kAccBias;
-                            const float d2 = __uint_as_float(y2[qq]) - kAccBias;
-                            const float d3 = __uint_as_float(y3[qq]) - kAccBias;
+                            // exact Y_i as floats (|Y| < 2^22: the integer add puts Y in
+                            // the mantissa of 1.5 * 2^23), then equation 10 and
+                            // equation 11's running sum
+                            const float d1 = __uint_as_float(y1[qq] + kAccBiasBits) - kAccBias;
+                            const float d2 = __uint_as_float(y2[qq] + kAccBiasBits) - kAccBias;
+                            const float d3 = __uint_as_float(y3[qq] + kAccBiasBits) - kAccBias;
                             const float v = fmaf(d3, kR3, fmaf(d2, kR2, d1));
                             acc[8 * c + qq] = fmaf(v, am[qq] * scc, acc[8 * c + qq]);
                         }
@@ -743,21 +747,15 @@ W4A16_ROLE_UNROLL
                                 const int m = tc.t0 + t;
                                 if (t < nt && m >= P.dbg_m0 && m < P.dbg_m1) {
                                     const size_t o = (static_cast<size_t>(m - P.dbg_m0) * P.G + grp) * wn + (n - P.dbg_n0);
-                                    P.dbg_yint[o] = static_cast<int32_t>(y1[qq] - kAccBiasBits);
-                                    P.dbg_yint[plane + o] = static_cast<int32_t>(y2[qq] - kAccBiasBits);
-                                    P.dbg_yint[2 * plane + o] = static_cast<int32_t>(y3[qq] - kAccBiasBits);
+                                    P.dbg_yint[o] = static_cast<int32_t>(y1[qq]);
+                                    P.dbg_yint[plane + o] = static_cast<int32_t>(y2[qq]);
+                                    P.dbg_yint[2 * plane + o] = static_cast<int32_t>(y3[qq]);
                                     if (n == P.dbg_n0)
                                         P.dbg_amax[static_cast<size_t>(m - P.dbg_m0) * P.G + grp] = am[qq];
                                 }
                             }
                         }
                     }
-                    // reset this group's columns to the bias
-#pragma unroll
-                    for (int rr = 0; rr < 3; ++rr)
-#pragma unroll
-                        for (int c = 0; c < TE / 8; ++c) tmem_st8_fill(b_addr + rr * TT + 8 * c, kAccBiasBits);
-                    tmem_st_wait();
                 } else {
 #pragma unroll
                     for (int c = 0; c < TE / 16; ++c) {
@@ -773,7 +771,19 @@ W4A16_ROLE_UNROLL
                 if (lane == 0) mbar_arrive(smem_addr(&accempty_bar[ab]));
                 if (warp == C::kEpiWarp0 && lane == 0 && j < 8) W4A16_TRACE_AT(44 + j);
             }
-            if (ok && P.splits == 1 && P.write_y && n_ok) {
+            if (C::kEpiRR) {
+                // groups 1..NEPI-1 hand their partial sums to group 0, which
+                // adds them in group order (deterministic)
+                if (eg > 0)
+#pragma unroll
+                    for (int t = 0; t < TE; ++t) rr_part[((eg - 1) * TT + t) * kBN + r] = acc[t];
+                named_bar_sync(1 + NEPI, C::kEpiThreads);
+                if (eg == 0)
+                    for (int e2 = 1; e2 < NEPI; ++e2)
+#pragma unroll
+                        for (int t = 0; t < TE; ++t) acc[t] += rr_part[((e2 - 1) * TT + t) * kBN + r];
+            }
+            if (ok && P.splits == 1 && P.write_y && n_ok && (!C::kEpiRR || eg == 0)) {
 #pragma unroll
                 for (int t = 0; t < TE; ++t)
                     if (tb + t < nt) P.y[static_cast<size_t>(tc.t0 + tb + t) * P.N + n] = __float2half_rn(acc[t]);
@@ -806,7 +816,7 @@ W4A16_ROLE_UNROLL
         // reduction buffer of the cluster rank that owns them: element
         // e = t * 128 + r belongs to rank e / per and lands in slot
         // [this rank][e - owner * per] there.
-        if (C::kRedBytes > 0 && P.splits > 1 && ok) {
+        if (C::kRedBytes > 0 && P.splits > 1 && ok && (!C::kEpiRR || eg == 0)) {
             const int S = P.splits;
             const int per = (TT * kBN + S - 1) / S;
             const uint32_t me = cluster_ctarank();
