@@ -275,12 +275,13 @@ w4a16_status launch_gemm(const CUtensorMap& map, const GemmParams& P, dim3 grid,
 // Kernel instances (variant, token tile, operand stages, weight stages,
 // converter groups, epilogue groups, MMA issuers, scale in the epilogue);
 // one CTA per SM, 512 Tensor Memory columns.
-//   decode (M <= 16): MSD <16, 8, 12, 2, 1, 4>   DEQUANT <16, 4, 12, 2, 1, 4, scale in epilogue>
-//     two converter groups and four MMA issuers: each small MMA (N = 48 / 16)
-//     holds its issuing thread for far longer than the tensor core needs, so
-//     the issue is spread over several warps
-//   larger M:         MSD <64, 4, 4, 1, 2, 1>   DEQUANT <128, 4, 4, 1, 1, 1>
-//     MSD's per-group combine is the bottleneck: two epilogue groups
+//   decode (M <= 16): MSD <16, 8, 12, 2, 2, 4>   DEQUANT <16, 4, 12, 2, 2, 4, scale in epilogue>
+//     four MMA issuers: each small MMA (N = 48 / 16) holds its issuing
+//     thread for far longer than the tensor core needs (two issuers with
+//     more operand stages measured 40 % slower); two epilogue groups take
+//     alternate K groups; 16 activation stages of their own
+//   larger M:         MSD <64, 4, 4, 2, 2, 1>   DEQUANT <128, 4, 4, 2, 1, 1>
+//     two converter groups; MSD's per-group combine needs two epilogue groups
 w4a16_status launch_for(int op, int TT, const CUtensorMap& map, const GemmParams& P, dim3 grid, cudaStream_t s)
 {
     if (op == W4A16_OP_MSD) {

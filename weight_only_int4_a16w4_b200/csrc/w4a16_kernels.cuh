@@ -102,8 +102,9 @@ struct GemmParams {
 
 // Compile-time shape of one gemm_kernel instance.
 //   TT     tokens per tile (MMA N for DEQUANT, N / 3 for MSD)
-//   ST     operand stages: stage s holds the activation tile of a chunk in
-//          shared memory and its converted A operand in Tensor Memory
+//   ST     operand stages: the converted A operand of a chunk in Tensor
+//          Memory (and, except on the decode tile, its activation tile in
+//          shared memory; the decode tile keeps 16 activation stages)
 //   WST    weight stages (shared memory only): the packed weight chunk and
 //          (optionally) its scale rows; deeper than ST so that enough weight
 //          bytes are in flight while Tensor Memory bounds ST
@@ -130,7 +131,11 @@ struct GemmCfg {
     static constexpr int kMmaN = kVals * TT;
     static constexpr int kBBytes = kIsMsd ? 3 * TT * 128 : 2 * TT * 128;   // activation tile per stage
     static constexpr int kSBytes = (kIsMsd || SEPI) ? 0 : 1024;            // up to 4 scale rows
-    static constexpr int kStage = kBBytes;                                 // operand stage (shared part)
+    static constexpr int kStage = kBBytes;                                 // activation stage (shared memory)
+    // activation stages: on the decode tile the tiles are small and every
+    // CTA reads the same ones from L2, so a deep ring of their own keeps the
+    // L2 latency off the MMA's path; elsewhere one per operand stage
+    static constexpr int kBST = TT == 16 ? 16 : ST;
     static constexpr int kWSlot = kWStage + kSBytes;                       // weight stage
     static constexpr int kMaxIssuers = NISS;
     static constexpr int kNBuf = kGroupAcc ? (NISS > 2 ? NISS : 2) : 1;
@@ -154,15 +159,16 @@ struct GemmCfg {
     static constexpr int kTokPerEpi = kEpiRR ? TT : TT / NEPI;
     static constexpr int kRedBytes = TT == 16 ? TT * kBN * 4 + 256 : 0;     // split-K partials (decode tile only)
     static constexpr int kRRBytes = kEpiRR ? (NEPI - 1) * TT * kBN * 4 : 0; // partial sums of groups 1..NEPI-1
-    static constexpr int kNumBars = 3 * ST + 2 * WST + 2 * kNBuf + kMaxIssuers;
-    static constexpr int kSmem = ST * kStage + WST * kWSlot + kRedBytes + kRRBytes + 1024 + 8 * kNumBars + 16 +
+    static constexpr int kNumBars = 2 * kBST + 2 * ST + 2 * WST + 2 * kNBuf + kMaxIssuers;
+    static constexpr int kSmem = kBST * kStage + WST * kWSlot + kRedBytes + kRRBytes + 1024 + 8 * kNumBars + 16 +
                                  2 * TT * 4 * NEPI + 16;
     static_assert(kColsUsed <= 512, "Tensor Memory overflow");
     static_assert(kMmaN % 16 == 0 && kMmaN >= 16 && kMmaN <= 256, "MMA N out of range");
     static_assert(TT % 16 == 0 && kTokPerEpi % 16 == 0, "token tile must split into 16-token pieces");
     static_assert(kStage % 1024 == 0 && kWSlot % 1024 == 0, "stages must keep 1024-byte alignment");
     static_assert(kSmem <= 227 * 1024, "shared memory overflow");
-    static_assert(ST % NCONV == 0 && ST % NISS == 0 && WST % NCONV == 0, "stages must split evenly over the groups");
+    static_assert(ST % NCONV == 0 && ST % NISS == 0 && WST % NCONV == 0 && kBST % NISS == 0,
+                  "stages must split evenly over the groups");
     static_assert(NISS == 1 || NISS == 2 || NISS == 4, "1, 2 or 4 MMA issuers");
     static_assert(!SEPI || !kIsMsd, "SEPI is a DEQUANT option");
     static_assert(!kEpiRR || (kGroupAcc && kNBuf % NEPI == 0), "round-robin epilogue needs per-group buffers");
@@ -377,12 +383,13 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
     using C = GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, SEPI>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* wsm = smem + ST * C::kStage;                              // weight slots
+    uint8_t* wsm = smem + C::kBST * C::kStage;                         // weight slots
     float* red = reinterpret_cast<float*>(wsm + WST * C::kWSlot);      // split-K partials pushed by the cluster
     float* rr_part = reinterpret_cast<float*>(wsm + WST * C::kWSlot + C::kRedBytes);   // [NEPI-1][TT][128]
     uint64_t* bars = reinterpret_cast<uint64_t*>(wsm + WST * C::kWSlot + C::kRedBytes + C::kRRBytes);
-    uint64_t* bfull_bar = bars;                 // [ST] activation tile landed
-    uint64_t* sfree_bar = bfull_bar + ST;       // [ST] operand stage free again (MMA done)
+    uint64_t* bfull_bar = bars;                 // [kBST] activation tile landed
+    uint64_t* bfree_bar = bfull_bar + C::kBST;  // [kBST] activation stage free again (MMA done)
+    uint64_t* sfree_bar = bfree_bar + C::kBST;  // [ST] operand stage free again (MMA done)
     uint64_t* afull_bar = sfree_bar + ST;       // [ST] A operand written to Tensor Memory
     uint64_t* wfull_bar = afull_bar + ST;       // [WST] weight slot landed
     uint64_t* wempty_bar = wfull_bar + WST;     // [WST] weight slot read by its converter group
@@ -412,8 +419,11 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
     const int grp0 = (kc0 * kKC) / P.g;                 // first group of this split
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < ST; ++s) {
+        for (int s = 0; s < C::kBST; ++s) {
             mbar_init(smem_addr(&bfull_bar[s]), 1);
+            mbar_init(smem_addr(&bfree_bar[s]), 1);
+        }
+        for (int s = 0; s < ST; ++s) {
             mbar_init(smem_addr(&sfree_bar[s]), 1);
             mbar_init(smem_addr(&afull_bar[s]), 4);
         }
@@ -456,9 +466,11 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
             const __half* ssrc = P.scale[tc.e];
             const uint32_t srow_bytes = static_cast<uint32_t>(min(kBN, P.N - n0)) * 2u;
             if (!weights) griddep_wait();
-            const int ring = weights ? WST : ST;
+            const int ring = weights ? WST : C::kBST;
             uint64_t* fullb = weights ? wfull_bar : bfull_bar;
-            uint64_t* freeb = weights ? wempty_bar : sfree_bar;
+            // with one activation stage per operand stage the MMA's stage
+            // commit frees both
+            uint64_t* freeb = weights ? wempty_bar : (C::kBST == ST ? sfree_bar : bfree_bar);
             int issued = 0;
             for (int i = 0; i < nchunks; ++i) {
                 const int s = i % ring;
@@ -525,12 +537,14 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
             for (int i = q; i < nchunks; i += issuers) {
                 const int s = i % ST;
                 const uint32_t ph = (i / ST) & 1;
+                const int bs = i % C::kBST;
+                const uint32_t bph = (i / C::kBST) & 1;
                 if (i == 2) W4A16_TRACE_AT(57);
                 if (!mbar_wait(smem_addr(&afull_bar[s]), ph, tmo, P.status, abort_flag)) break;
-                if (!mbar_wait(smem_addr(&bfull_bar[s]), ph, tmo, P.status, abort_flag)) break;
+                if (!mbar_wait(smem_addr(&bfull_bar[bs]), bph, tmo, P.status, abort_flag)) break;
                 if (i == 2) W4A16_TRACE_AT(58);
                 tc_fence_after();
-                const uint64_t bdesc = smem_desc_sw128(smem_addr(smem + s * C::kStage));
+                const uint64_t bdesc = smem_desc_sw128(smem_addr(smem + bs * C::kStage));
                 const uint32_t a_base = tmem_a0 + s * C::kACols;
                 const int kc = kc0 + i;
                 const int nsteps = min(kSteps, (P.K - kc * kKC) / kStepK);   // K-padding steps are skipped
@@ -574,6 +588,7 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
                 if (lane == 0) {
                     if (i < 8) W4A16_TRACE_AT(28 + i);
                     tc_commit(smem_addr(&sfree_bar[s]));
+                    if (C::kBST != ST) tc_commit(smem_addr(&bfree_bar[bs]));
                 }
                 __syncwarp();
                 first_chunk = false;
