@@ -280,8 +280,9 @@ w4a16_status launch_gemm(const CUtensorMap& map, const GemmParams& P, dim3 grid,
 //     thread for far longer than the tensor core needs (two issuers with
 //     more operand stages measured 40 % slower); two epilogue groups take
 //     alternate K groups; 16 activation stages of their own
-//   larger M:         MSD <64, 4, 4, 2, 2, 1>   DEQUANT <128, 4, 4, 2, 1, 1>
-//     two converter groups; MSD's per-group combine needs two epilogue groups
+//   larger M:         MSD <64, 4, 4, 2, 2, 1>   DEQUANT <128, 4, 4, 2, 1, 2>
+//     two converter groups; MSD's per-group combine needs two epilogue
+//     groups; DEQUANT two issuers, each into its own accumulator
 w4a16_status launch_for(int op, int TT, const CUtensorMap& map, const GemmParams& P, dim3 grid, cudaStream_t s)
 {
     if (op == W4A16_OP_MSD) {
@@ -294,7 +295,7 @@ w4a16_status launch_for(int op, int TT, const CUtensorMap& map, const GemmParams
         return launch_gemm<kMsd, 64, 4, 4, 2, 2, 1, false>(map, P, grid, s);
     }
     if (TT == 16) return launch_gemm<kDeq, 16, 4, 12, 2, 2, 4, true>(map, P, grid, s);
-    return launch_gemm<kDeq, 128, 4, 4, 2, 1, 1, false>(map, P, grid, s);
+    return launch_gemm<kDeq, 128, 4, 4, 2, 1, 2, false>(map, P, grid, s);
 }
 
 template <int VPL>
@@ -335,7 +336,7 @@ w4a16_status launch_expand(const void* x, int M, int K, int g, int8_t* xq, float
     return W4A16_OK;
 }
 
-void base_params(GemmParams& P, int M, int K, int N, int g, const Shape& s, void* ws)
+void base_params(GemmParams& P, int op, int M, int K, int N, int g, const Shape& s, void* ws)
 {
     std::memset(&P, 0, sizeof(P));
     P.M = M;
@@ -349,7 +350,8 @@ void base_params(GemmParams& P, int M, int K, int N, int g, const Shape& s, void
     P.splits = s.splits;
     P.unit = s.unit;
     P.E = 1;
-    P.issuers = 1;
+    // the large DEQUANT tile has one accumulator per MMA issuer (two)
+    P.issuers = (op == W4A16_OP_DEQUANT && s.TT != 16) ? 2 : 1;
     P.status = static_cast<uint32_t*>(ws);
     P.timeout_ns = g_timeout_ns.load();
     P.write_y = 1;
@@ -469,7 +471,7 @@ w4a16_status dense_matmul(int op, const void* x, const void* w_packed, const voi
     if (ws_bytes < full.total) return W4A16_ERR_WORKSPACE;
 
     GemmParams P;
-    base_params(P, M, K, N, g, s, ws);
+    base_params(P, op, M, K, N, g, s, ws);
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     P.w[0] = static_cast<const uint8_t*>(w_packed);
     P.scale[0] = static_cast<const __half*>(scale);
@@ -627,7 +629,7 @@ w4a16_status w4a16_grouped_matmul(int op, const void* x, const void* const* w_pa
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
 
     GemmParams P;
-    base_params(P, T, K, N, group_size, s, workspace);
+    base_params(P, op, T, K, N, group_size, s, workspace);
     uint8_t* wsb = static_cast<uint8_t*>(workspace);
     P.E = E;
     P.offsets = offsets;

@@ -138,7 +138,10 @@ struct GemmCfg {
     static constexpr int kBST = TT == 16 ? 16 : ST;
     static constexpr int kWSlot = kWStage + kSBytes;                       // weight stage
     static constexpr int kMaxIssuers = NISS;
-    static constexpr int kNBuf = kGroupAcc ? (NISS > 2 ? NISS : 2) : 1;
+    // accumulator buffers: per group (two, or one per issuer); a single
+    // accumulator over all of K otherwise, one per issuer (added up, in
+    // issuer order, by the epilogue)
+    static constexpr int kNBuf = kGroupAcc ? (NISS > 2 ? NISS : 2) : NISS;
     static constexpr int kAccStride = ((kMmaN + 31) / 32) * 32;
     static constexpr int kAccCols = kNBuf * kAccStride;
     static constexpr int kACols = kIsMsd ? 32 : 64;                        // A operand per stage
@@ -581,7 +584,9 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
                         }
                         __syncwarp();
                     } else {
-                        if (lane == 0) mma_f16_ts(tmem, a_base + 8 * j, bd, idesc, (first_chunk && j == 0) ? 0u : 1u);
+                        if (lane == 0)
+                            mma_f16_ts(tmem + q * C::kAccStride, a_base + 8 * j, bd, idesc,
+                                       (first_chunk && j == 0) ? 0u : 1u);
                         __syncwarp();
                     }
                 }
@@ -595,7 +600,7 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
                 if (failed) break;
             }
             if (lane == 0) {
-                if (!C::kGroupAcc) tc_commit(smem_addr(&accfull_bar[0]));
+                if (!C::kGroupAcc) tc_commit(smem_addr(&accfull_bar[q]));
                 // Every MMA issued has completed before Tensor Memory is freed.
                 tc_commit(smem_addr(&done_bar[q]));
             }
@@ -804,23 +809,38 @@ W4A16_ROLE_UNROLL
                     if (tb + t < nt) P.y[static_cast<size_t>(tc.t0 + tb + t) * P.N + n] = __float2half_rn(acc[t]);
             }
         } else {
-            // one accumulator over all of K (scales applied by the converter)
+            // one accumulator over all of K per issuer (scales applied by the
+            // converter); issuers with no chunk left theirs unwritten
             griddep_wait();
-            ok = nchunks > 0 && mbar_wait(smem_addr(&accfull_bar[0]), 0, tmo, P.status, abort_flag);
+            const int nacc = min(issuers, nchunks);
+            ok = nchunks > 0;
+            for (int q = 0; q < nacc && ok; ++q)
+                ok = mbar_wait(smem_addr(&accfull_bar[q]), 0, tmo, P.status, abort_flag);
             if (ok) {
                 if (warp == C::kEpiWarp0 && lane == 0) W4A16_TRACE_AT(36);
                 tc_fence_after();
 #pragma unroll 1
                 for (int c = 0; c < TE / 16; ++c) {
-                    uint32_t u[16];
-                    tmem_ld16(t_addr + tb + 16 * c, u);
-                    tmem_ld_wait();
+                    float v[16];
+                    {
+                        uint32_t u[16];
+                        tmem_ld16(t_addr + tb + 16 * c, u);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(u[k]);
+                    }
+                    for (int q = 1; q < nacc; ++q) {
+                        uint32_t u[16];
+                        tmem_ld16(t_addr + q * C::kAccStride + tb + 16 * c, u);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) v[k] += __uint_as_float(u[k]);
+                    }
                     if (P.write_y && n_ok) {
 #pragma unroll
                         for (int k = 0; k < 16; ++k)
                             if (tb + 16 * c + k < nt)
-                                P.y[static_cast<size_t>(tc.t0 + tb + 16 * c + k) * P.N + n] =
-                                    __float2half_rn(__uint_as_float(u[k]));
+                                P.y[static_cast<size_t>(tc.t0 + tb + 16 * c + k) * P.N + n] = __float2half_rn(v[k]);
                     }
                 }
                 tc_fence_before();
