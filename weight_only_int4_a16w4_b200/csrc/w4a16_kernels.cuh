@@ -164,7 +164,7 @@ struct GemmCfg {
     static constexpr int kRRBytes = kEpiRR ? (NEPI - 1) * TT * kBN * 4 : 0; // partial sums of groups 1..NEPI-1
     static constexpr int kNumBars = 2 * kBST + 2 * ST + 2 * WST + 2 * kNBuf + kMaxIssuers;
     static constexpr int kSmem = kBST * kStage + WST * kWSlot + kRedBytes + kRRBytes + 1024 + 8 * kNumBars + 16 +
-                                 2 * TT * 4 * NEPI + 16;
+                                 4 * NEPI * 2 * TT * 4 + 16;
     static_assert(kColsUsed <= 512, "Tensor Memory overflow");
     static_assert(kMmaN % 16 == 0 && kMmaN >= 16 && kMmaN <= 256, "MMA N out of range");
     static_assert(TT % 16 == 0 && kTokPerEpi % 16 == 0, "token tile must split into 16-token pieces");
@@ -401,8 +401,9 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
     uint64_t* done_bar = accempty_bar + C::kNBuf;    // [kMaxIssuers] all MMAs of an issuer completed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + C::kMaxIssuers);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    // [NEPI][2][TT] floats read as float4: round up to a 16-byte boundary
-    // (the barriers before it end on an 8-byte boundary only)
+    // A_max ring, one per epilogue warp: [4 * NEPI][2][TT] floats read as
+    // float4: round up to a 16-byte boundary (the barriers before it end on
+    // an 8-byte boundary only)
     float* amax_sm = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(tmem_slot + 4) + 15) & ~uintptr_t(15));
 
     TileCoord tc;
@@ -685,8 +686,6 @@ W4A16_ROLE_UNROLL
     } else if (warp >= C::kEpiWarp0) {
         // ============================ epilogue ============================
         const int eg = (warp - C::kEpiWarp0) >> 2;             // epilogue group
-        // thread index within the threads that share the A_max ring
-        const int et = threadIdx.x - 32 * (C::kEpiRR ? C::kEpiWarp0 + 4 * eg : C::kEpiWarp0);
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32);
         const int r = lane_base + lane;
         const int n = n0 + r;
@@ -711,25 +710,43 @@ W4A16_ROLE_UNROLL
             const int ngroups = min(kc1 * kKC, P.K) / P.g - grp0;
             const __half* sc_e = P.scale[tc.e];
             const int jstep = C::kEpiRR ? NEPI : 1, j0 = C::kEpiRR ? eg : 0;
-            float am_next = 0.f, sc_next = 0.f;
-            if (j0 < ngroups) {
-                if (C::kIsMsd && et < nt) am_next = __ldg(P.amax + static_cast<size_t>(grp0 + j0) * P.M + tc.t0 + et);
-                if (n_ok && sc_e) sc_next = __half2float(sc_e[static_cast<size_t>(grp0 + j0) * P.N + n]);
+            // A_max of the tile's TT tokens for the next group, lane l holding
+            // tokens l, l + 32, ...; each warp keeps its own two-slot ring in
+            // shared memory, so only the warp synchronises
+            constexpr int AMV = (TT + 31) / 32;
+            float am_next[AMV];
+            float sc_next = 0.f;
+#pragma unroll
+            for (int v = 0; v < AMV; ++v) {
+                const int tok = lane + 32 * v;
+                am_next[v] = (C::kIsMsd && j0 < ngroups && tok < nt)
+                                 ? __ldg(P.amax + static_cast<size_t>(grp0 + j0) * P.M + tc.t0 + tok) : 0.f;
             }
+            if (j0 < ngroups && n_ok && sc_e) sc_next = __half2float(sc_e[static_cast<size_t>(grp0 + j0) * P.N + n]);
+            float* am_ring = amax_sm + (warp - C::kEpiWarp0) * 2 * TT;
             for (int j = j0, jj = 0; j < ngroups; j += jstep, ++jj) {
                 const int grp = grp0 + j;
                 const int ab = j % C::kNBuf;
                 const uint32_t abph = (j / C::kNBuf) & 1;
-                float* am_slot = amax_sm + ((C::kEpiRR ? eg : 0) * 2 + (jj & 1)) * TT;
-                if (C::kIsMsd && et < TT) am_slot[et] = am_next;
+                float* am_slot = am_ring + (jj & 1) * TT;
+                if (C::kIsMsd) {
+#pragma unroll
+                    for (int v = 0; v < AMV; ++v)
+                        if (lane + 32 * v < TT) am_slot[lane + 32 * v] = am_next[v];
+                }
                 const float sc = sc_next;
                 if (j + jstep < ngroups) {       // prefetch the next group's A_max and scale
-                    if (C::kIsMsd)
-                        am_next = (et < nt) ? __ldg(P.amax + static_cast<size_t>(grp + jstep) * P.M + tc.t0 + et) : 0.f;
+                    if (C::kIsMsd) {
+#pragma unroll
+                        for (int v = 0; v < AMV; ++v) {
+                            const int tok = lane + 32 * v;
+                            am_next[v] =
+                                tok < nt ? __ldg(P.amax + static_cast<size_t>(grp + jstep) * P.M + tc.t0 + tok) : 0.f;
+                        }
+                    }
                     if (n_ok && sc_e) sc_next = __half2float(sc_e[static_cast<size_t>(grp + jstep) * P.N + n]);
                 }
-                // every thread that shares the A_max ring, every group
-                if (C::kIsMsd) named_bar_sync(1 + (C::kEpiRR ? eg : 0), C::kEpiRR ? 128 : C::kEpiThreads);
+                if (C::kIsMsd) __syncwarp();
                 if (ok && !mbar_wait(smem_addr(&accfull_bar[ab]), abph, tmo, P.status, abort_flag)) ok = false;
                 if (!ok) continue;
                 if (warp == C::kEpiWarp0 && lane == 0 && j < 8) W4A16_TRACE_AT(36 + j);
