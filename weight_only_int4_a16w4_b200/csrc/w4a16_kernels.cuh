@@ -527,7 +527,10 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
         // per chunk frees the operand stage for both.  The warp runs
         // converged; lane 0 issues the MMAs and commits.
         const int q = warp - 2;
-        if (q < issuers) {
+        // One lane runs the issuer's whole loop (waits, MMAs, commits): a warp
+        // that reconverges after every MMA roughly doubles the issue cost of
+        // each one.
+        if (q < issuers && lane == 0) {
             constexpr uint32_t idesc = C::kIsMsd ? idesc_s8_s32(C::kMmaN) : idesc_f16_f32(C::kMmaN);
             constexpr int kSteps = C::kIsMsd ? 4 : 8;         // MMA K steps per 128-deep chunk
             constexpr int kStepK = kKC / kSteps;
@@ -576,36 +579,25 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
                             tc_fence_after();
                         }
                         const uint32_t d = tmem + ab * C::kAccStride;
-                        if (lane == 0) {
-                            // a group's first K step overwrites the buffer
-                            if (C::kIsMsd) mma_i8_ts(d, a_base + 8 * j, bd, idesc, gpos == 0 ? 0u : 1u);
-                            else mma_f16_ts(d, a_base + 8 * j, bd, idesc, gpos == 0 ? 0u : 1u);
-                            if (i == 2 && j < 4) W4A16_TRACE_AT(60 + j);
-                            if (gpos == gsteps - 1) tc_commit(smem_addr(&accfull_bar[ab]));
-                        }
-                        __syncwarp();
+                        // a group's first K step overwrites the buffer
+                        if (C::kIsMsd) mma_i8_ts(d, a_base + 8 * j, bd, idesc, gpos == 0 ? 0u : 1u);
+                        else mma_f16_ts(d, a_base + 8 * j, bd, idesc, gpos == 0 ? 0u : 1u);
+                        if (i == 2 && j < 4) W4A16_TRACE_AT(60 + j);
+                        if (gpos == gsteps - 1) tc_commit(smem_addr(&accfull_bar[ab]));
                     } else {
-                        if (lane == 0)
-                            mma_f16_ts(tmem + q * C::kAccStride, a_base + 8 * j, bd, idesc,
-                                       (first_chunk && j == 0) ? 0u : 1u);
-                        __syncwarp();
+                        mma_f16_ts(tmem + q * C::kAccStride, a_base + 8 * j, bd, idesc,
+                                   (first_chunk && j == 0) ? 0u : 1u);
                     }
                 }
-                if (lane == 0) {
-                    if (i < 8) W4A16_TRACE_AT(28 + i);
-                    tc_commit(smem_addr(&sfree_bar[s]));
-                    if (C::kBST != ST) tc_commit(smem_addr(&bfree_bar[bs]));
-                }
-                __syncwarp();
+                if (i < 8) W4A16_TRACE_AT(28 + i);
+                tc_commit(smem_addr(&sfree_bar[s]));
+                if (C::kBST != ST) tc_commit(smem_addr(&bfree_bar[bs]));
                 first_chunk = false;
                 if (failed) break;
             }
-            if (lane == 0) {
-                if (!C::kGroupAcc) tc_commit(smem_addr(&accfull_bar[q]));
-                // Every MMA issued has completed before Tensor Memory is freed.
-                tc_commit(smem_addr(&done_bar[q]));
-            }
-            __syncwarp();
+            if (!C::kGroupAcc) tc_commit(smem_addr(&accfull_bar[q]));
+            // Every MMA issued has completed before Tensor Memory is freed.
+            tc_commit(smem_addr(&done_bar[q]));
             mbar_wait(smem_addr(&done_bar[q]), 0, tmo, P.status, nullptr);
         }
         __syncwarp();
