@@ -557,6 +557,27 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
                 const int nsteps = min(kSteps, (P.K - kc * kKC) / kStepK);   // K-padding steps are skipped
                 const int step0 = i * kSteps;        // K step index from the split's first group boundary
                 bool failed = false;
+                if (C::kGroupAcc && gsteps == kSteps && nsteps == kSteps) {
+                    // a group is exactly this chunk (g = 128): buffer i % NBUF,
+                    // every step's operands and flags known at compile time
+                    const int ab = i % C::kNBuf;
+                    if (!mbar_wait(smem_addr(&accempty_bar[ab]), (i / C::kNBuf) & 1, tmo, P.status, abort_flag))
+                        break;
+                    tc_fence_after();
+                    const uint32_t d = tmem + ab * C::kAccStride;
+#pragma unroll
+                    for (int j = 0; j < kSteps; ++j) {
+                        const uint64_t bd =
+                            C::kIsMsd ? bdesc + 2 * j : bdesc + ((j >> 2) * (TT * 128) >> 4) + 2 * (j & 3);
+                        if (C::kIsMsd) mma_i8_ts(d, a_base + 8 * j, bd, idesc, j == 0 ? 0u : 1u);
+                        else mma_f16_ts(d, a_base + 8 * j, bd, idesc, j == 0 ? 0u : 1u);
+                    }
+                    tc_commit(smem_addr(&accfull_bar[ab]));
+                    tc_commit(smem_addr(&sfree_bar[s]));
+                    if (C::kBST != ST) tc_commit(smem_addr(&bfree_bar[bs]));
+                    first_chunk = false;
+                    continue;
+                }
 #pragma unroll
                 for (int j = 0; j < kSteps; ++j) {
                     if (j >= nsteps) break;
