@@ -302,8 +302,22 @@ __global__ void __launch_bounds__(256) expand_kernel(const __half* __restrict__ 
     const size_t base = static_cast<size_t>(m) * K + static_cast<size_t>(gi) * g + lane * VPL;
 
     float v[VPL];
+    if constexpr (VPL % 4 == 0) {
+        // 8-byte loads (VPL consecutive halves, 8-byte aligned: K % 32 == 0)
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) v[i] = __half2float(x[base + i]);
+        for (int i = 0; i < VPL; i += 4) {
+            const uint2 raw = *reinterpret_cast<const uint2*>(x + base + i);
+            const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+            const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+            v[i] = lo.x;
+            v[i + 1] = lo.y;
+            v[i + 2] = hi.x;
+            v[i + 3] = hi.y;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) v[i] = __half2float(x[base + i]);
+    }
     float am = 0.f;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) am = fmaxf(am, fabsf(v[i]));
@@ -328,11 +342,28 @@ __global__ void __launch_bounds__(256) expand_kernel(const __half* __restrict__ 
         }
     }
     const size_t plane = static_cast<size_t>(M) * K;
+    if constexpr (VPL % 4 == 0) {
+        // one 4-byte store per plane and 4 digits (4-byte aligned)
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-        xq[base + i] = d1[i];
-        xq[plane + base + i] = d2[i];
-        xq[2 * plane + base + i] = d3[i];
+        for (int i = 0; i < VPL; i += 4) {
+            uint32_t w1 = 0, w2 = 0, w3 = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                w1 |= (static_cast<uint32_t>(static_cast<uint8_t>(d1[i + e]))) << (8 * e);
+                w2 |= (static_cast<uint32_t>(static_cast<uint8_t>(d2[i + e]))) << (8 * e);
+                w3 |= (static_cast<uint32_t>(static_cast<uint8_t>(d3[i + e]))) << (8 * e);
+            }
+            *reinterpret_cast<uint32_t*>(xq + base + i) = w1;
+            *reinterpret_cast<uint32_t*>(xq + plane + base + i) = w2;
+            *reinterpret_cast<uint32_t*>(xq + 2 * plane + base + i) = w3;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+            xq[base + i] = d1[i];
+            xq[plane + base + i] = d2[i];
+            xq[2 * plane + base + i] = d3[i];
+        }
     }
     if (lane == 0) amax[static_cast<size_t>(gi) * M + m] = am;
 }
