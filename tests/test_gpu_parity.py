@@ -195,11 +195,12 @@ def test_repeat_calls_are_deterministic(cuda_lib):
     torch.cuda.synchronize()
 
 
-# ---------------------------------------------------------------- decode GEMV (M <= 4)
+# ---------------------------------------------------------------- decode GEMVs
 
-# Shapes for the CUDA-core decode kernel: every group size, ragged N and K,
-# and work splits where many CTAs share one column tile (N small, K long) or
-# one CTA spans two tiles (N large, K short).
+# Small-M shapes (the CUDA-core GEMV, the warp-MMA GEMV or the decode tile,
+# whichever the dispatch picks): every group size, ragged N and K, and work
+# splits where many CTAs share one column tile (N small, K long) or one CTA
+# spans two tiles (N large, K short).
 GEMV = [
     # (M, K, N, g)                       what it covers
     (1, 4096, 136, 128),                 # 2 tiles x 32 chunks: ~32 CTAs add into each tile
@@ -258,6 +259,48 @@ def test_decode_shapes_both_variants(cuda_lib, M, K, N, g):
                      f"decode msd {M}x{K}x{N} g{g}")
     assert_deq_close(run_dense(w4, w4.OP_DEQUANT, c, dev), oracle.dequant(c.x, c.wp[0], c.scale[0], g),
                      f"decode dequant {M}x{K}x{N} g{g}")
+
+
+# Shapes that take the warp-MMA GEMV (dequant: g % 128 == 0, M <= 8; MSD:
+# M <= 2 and K >= 2N): rows up to the full lower half of the m16 tile,
+# quads fewer than warps (idle warps), groups of 2-4 quads cut by the
+# warps' K split, one column block per CTA, a CTA with several 4-block
+# rounds and a ragged last one, a single 8-column block.
+MMA_DEQ = [
+    # (M, K, N, g)
+    (5, 4096, 520, 128),
+    (8, 1536, 264, 256),
+    (3, 1152, 776, 384),
+    (6, 2560, 14344, 512),
+    (2, 128, 64, 128),
+    (7, 8192, 8, 128),
+]
+MMA_MSD = [
+    (1, 8192, 1024, 128),
+    (2, 4096, 264, 256),
+    (2, 3072, 136, 384),
+    (1, 4096, 2048, 512),
+    (2, 1152, 8, 128),
+]
+
+
+@pytest.mark.parametrize("M,K,N,g", MMA_DEQ)
+def test_mma_gemv_dequant(cuda_lib, M, K, N, g):
+    w4 = cuda_lib
+    c = make_case(M, K, N, g, seed=M * 313 + K * 17 + N * 5 + g)
+    dev = upload(w4, c)
+    assert_deq_close(run_dense(w4, w4.OP_DEQUANT, c, dev), oracle.dequant(c.x, c.wp[0], c.scale[0], g),
+                     f"mma dequant {M}x{K}x{N} g{g}")
+
+
+@pytest.mark.parametrize("M,K,N,g", MMA_MSD)
+def test_mma_gemv_msd(cuda_lib, M, K, N, g):
+    w4 = cuda_lib
+    c = make_case(M, K, N, g, seed=M * 317 + K * 19 + N * 3 + g)
+    c.x[M - 1, g:2 * g] = 0              # an all-zero group
+    dev = upload(w4, c)
+    assert_msd_close(run_dense(w4, w4.OP_MSD, c, dev), oracle.msd(c.x, c.wp[0], c.scale[0], g),
+                     f"mma msd {M}x{K}x{N} g{g}")
 
 
 def test_gemv_repeat_calls_are_deterministic(cuda_lib):

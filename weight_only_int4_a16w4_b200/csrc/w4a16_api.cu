@@ -14,6 +14,7 @@
 
 #include "../../include/w4a16.h"
 #include "w4a16_gemv.cuh"
+#include "w4a16_gemv_mma.cuh"
 #include "w4a16_kernels.cuh"
 
 using namespace w4a16;
@@ -155,31 +156,68 @@ Shape grouped_shape(int op, int T, int K, int N, int g, int E)
 
 // ---------------------------------------------------------------- the CUDA-core decode GEMV
 
-// Largest M that takes the GEMV (w4a16_gemv.cuh) instead of the tensor-core
-// decode tile; W4A16_GEMV_MAX_M overrides it (0 turns the GEMV off).
-int gemv_max_m(int op)
+int gemv_mma_rows(int op, int M)
 {
-    static int v[2] = {-1, -1};
-    if (v[op] < 0) {
-        const char* e = std::getenv("W4A16_GEMV_MAX_M");
-        int d = 4;
-        if (e && *e) d = std::atoi(e);
-        v[op] = std::max(0, std::min(d, 4));
+    if (op == W4A16_OP_MSD) return M <= 1 ? 1 : 2;
+    return M <= 1 ? 1 : (M <= 2 ? 2 : (M <= 4 ? 4 : 8));
+}
+
+int gemv_mma_smem(int op, int M, int K, int g)
+{
+    const int np = K / 32, ppg = g / 32;
+    // the shared-memory size does not depend on the row template argument
+    return op == W4A16_OP_MSD ? MgCfg<kMsd, 1>::smem_bytes(M, np, ppg) : MgCfg<kDeq, 1>::smem_bytes(M, np, ppg);
+}
+
+// The kernel of a dense call with a handful of rows.  Measured on B200
+// (consecutive dependent calls, weights streamed from HBM):
+//  * dequant, g % 128 == 0, M <= 8: the warp-MMA GEMV (w4a16_gemv_mma.cuh)
+//    beats the CUDA-core GEMV and the tensor-core decode tile at every size;
+//  * MSD, M == 1, up to 16 MB of weights: the CUDA-core GEMV
+//    (w4a16_gemv.cuh) -- at this size the call is a chain of two dependent
+//    kernels and the GEMV's own arithmetic is short;
+//  * MSD, M <= 2, K >= 2N: the warp-MMA GEMV;
+//  * g < 128 and M <= 4: the CUDA-core GEMV (the tensor tile is weak there);
+//  * everything else: the tensor-core decode tile.
+// W4A16_SMALL = tensor | cuda | mma forces one of them where it applies.
+enum SmallKernel { kSmallNone = 0, kSmallCuda = 1, kSmallMma = 2 };
+
+int small_override()
+{
+    static int v = -2;
+    if (v == -2) {
+        const char* e = std::getenv("W4A16_SMALL");
+        v = -1;
+        if (e && std::strcmp(e, "tensor") == 0) v = kSmallNone;
+        if (e && std::strcmp(e, "cuda") == 0) v = kSmallCuda;
+        if (e && std::strcmp(e, "mma") == 0) v = kSmallMma;
     }
-    return v[op];
+    return v;
 }
 
-bool use_gemv(int op, int M, int K, int E)
+int small_kernel(int op, int M, int K, int N, int g, int E)
 {
-    return E == 1 && M >= 1 && M <= gemv_max_m(op) && static_cast<long long>(M) * K <= kGemvMaxMK;
+    if (E != 1 || M < 1) return kSmallNone;
+    const bool mma_ok = g % 128 == 0 && M <= (op == W4A16_OP_MSD ? 2 : 8) &&
+                        gemv_mma_smem(op, M, K, g) <= kMaxSmemOptin;
+    const bool cuda_ok = M <= 4 && static_cast<long long>(M) * K <= kGemvMaxMK;
+    const int forced = small_override();
+    if (forced == kSmallNone) return kSmallNone;
+    if (forced == kSmallCuda) return cuda_ok ? kSmallCuda : kSmallNone;
+    if (forced == kSmallMma) return mma_ok ? kSmallMma : kSmallNone;
+    if (op == W4A16_OP_DEQUANT) return mma_ok ? kSmallMma : (cuda_ok ? kSmallCuda : kSmallNone);
+    if (cuda_ok && M == 1 && (g % 128 != 0 || static_cast<long long>(K) * N <= (32ll << 20))) return kSmallCuda;
+    if (mma_ok && K >= 2 * N) return kSmallMma;
+    if (cuda_ok && g % 128 != 0) return kSmallCuda;
+    return kSmallNone;
 }
 
-// CTAs of the GEMV: one per SM at most, never more than there are 32-column
+// CTAs of a GEMV: one per SM at most, never more than there are column
 // blocks.
 int gemv_ctas(int nblk) { return std::min(nblk, sm_count()); }
 
 struct WsLayout {
-    size_t xq = 0, amax = 0, rec = 0, rec_amax = 0, total = 0;
+    size_t xq = 0, amax = 0, rec = 0, total = 0;
 };
 
 WsLayout ws_layout(int op, const Shape& s, int M, int K, int N, int g, int E = 1)
@@ -193,12 +231,10 @@ WsLayout ws_layout(int op, const Shape& s, int M, int K, int N, int g, int E = 1
         off += align256(static_cast<size_t>(3) * M * K);
         L.amax = off;
         off += align256(static_cast<size_t>(K / g) * M * 4);
-        if (use_gemv(op, M, K, E)) {
-            // the decode GEMV's digit records [K/32][M][28 words] and A_max [M][K/g]
+        if (small_kernel(op, M, K, N, g, E) != kSmallNone) {
+            // the decode GEMV's digit records [K/32][M][28 words]
             L.rec = off;
             off += align256(static_cast<size_t>(K / 32) * M * kGemvRecWords * 4);
-            L.rec_amax = off;
-            off += align256(static_cast<size_t>(K / g) * M * 4);
         }
     }
     L.total = off;
@@ -387,8 +423,37 @@ w4a16_status launch_gemv_mr(const GemvParams& P, cudaStream_t stream)
     return W4A16_OK;
 }
 
+template <int VAR, int MR>
+w4a16_status launch_gemv_mma_mr(const GemvParams& P, cudaStream_t stream)
+{
+    auto kern = gemv_mma_kernel<VAR, MR>;
+    const int smem = gemv_mma_smem(VAR == kMsd ? W4A16_OP_MSD : W4A16_OP_DEQUANT, P.M, P.K, P.g);
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [&] {
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmemOptin);
+    });
+    if (attr_err != cudaSuccess) return W4A16_ERR_CUDA;
+    if (smem > kMaxSmemOptin) return W4A16_ERR_UNSUPPORTED;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(P.ctas), 1, 1);
+    cfg.blockDim = dim3(kMgThreads, 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = use_pdl() ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, kern, P) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return W4A16_ERR_CUDA;
+    }
+    return W4A16_OK;
+}
+
 template <int NSUB>
-cudaError_t launch_gemv_expand_n(const __half* x, int M, int K, int g, uint32_t* rec, float* amax, cudaStream_t s)
+cudaError_t launch_gemv_expand_n(const __half* x, int M, int K, int g, uint32_t* rec, cudaStream_t s)
 {
     const int span = NSUB * kKC;
     const long long warps = static_cast<long long>(M) * ((K + span - 1) / span);
@@ -401,11 +466,11 @@ cudaError_t launch_gemv_expand_n(const __half* x, int M, int K, int g, uint32_t*
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = use_pdl() ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, gemv_expand_kernel<NSUB>, x, M, K, g, rec, amax);
+    return cudaLaunchKernelEx(&cfg, gemv_expand_kernel<NSUB>, x, M, K, g, rec);
 }
 
-w4a16_status launch_gemv(int op, const void* x, const void* w_packed, const void* scale, int M, int K, int N, int g,
-                         void* y, void* ws, const Shape& s, const WsLayout& L, cudaStream_t stream)
+w4a16_status launch_gemv(int op, bool mma, const void* x, const void* w_packed, const void* scale, int M, int K, int N,
+                         int g, void* y, void* ws, const Shape& s, const WsLayout& L, cudaStream_t stream)
 {
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     GemvParams P;
@@ -421,29 +486,37 @@ w4a16_status launch_gemv(int op, const void* x, const void* w_packed, const void
     P.G = K / g;
     P.kchunks = s.kchunks;
     P.npieces = K / 32;
-    P.nblk = cdiv(N, 32);
+    P.nblk = mma ? N / 8 : cdiv(N, 32);
     P.ctas = gemv_ctas(P.nblk);
     if (op == W4A16_OP_MSD) {
         uint32_t* rec = reinterpret_cast<uint32_t*>(wsb + L.rec);
-        float* amax = reinterpret_cast<float*>(wsb + L.rec_amax);
         P.rec = rec;
-        P.amax = amax;
         const __half* xh = static_cast<const __half*>(x);
         cudaError_t e;
         switch (std::max(1, g / kKC)) {
-            case 1: e = launch_gemv_expand_n<1>(xh, M, K, g, rec, amax, stream); break;
-            case 2: e = launch_gemv_expand_n<2>(xh, M, K, g, rec, amax, stream); break;
-            case 3: e = launch_gemv_expand_n<3>(xh, M, K, g, rec, amax, stream); break;
-            case 4: e = launch_gemv_expand_n<4>(xh, M, K, g, rec, amax, stream); break;
+            case 1: e = launch_gemv_expand_n<1>(xh, M, K, g, rec, stream); break;
+            case 2: e = launch_gemv_expand_n<2>(xh, M, K, g, rec, stream); break;
+            case 3: e = launch_gemv_expand_n<3>(xh, M, K, g, rec, stream); break;
+            case 4: e = launch_gemv_expand_n<4>(xh, M, K, g, rec, stream); break;
             default: return W4A16_ERR_UNSUPPORTED;
         }
         if (e != cudaSuccess) {
             (void)cudaGetLastError();
             return W4A16_ERR_CUDA;
         }
+        if (mma) return gemv_mma_rows(op, M) == 1 ? launch_gemv_mma_mr<kMsd, 1>(P, stream)
+                                                  : launch_gemv_mma_mr<kMsd, 2>(P, stream);
         if (M == 1) return launch_gemv_mr<kMsd, 1>(P, stream);
         if (M == 2) return launch_gemv_mr<kMsd, 2>(P, stream);
         return launch_gemv_mr<kMsd, 4>(P, stream);
+    }
+    if (mma) {
+        switch (gemv_mma_rows(op, M)) {
+            case 1: return launch_gemv_mma_mr<kDeq, 1>(P, stream);
+            case 2: return launch_gemv_mma_mr<kDeq, 2>(P, stream);
+            case 4: return launch_gemv_mma_mr<kDeq, 4>(P, stream);
+            default: return launch_gemv_mma_mr<kDeq, 8>(P, stream);
+        }
     }
     if (M == 1) return launch_gemv_mr<kDeq, 1>(P, stream);
     if (M == 2) return launch_gemv_mr<kDeq, 2>(P, stream);
@@ -485,7 +558,10 @@ w4a16_status dense_matmul(int op, const void* x, const void* w_packed, const voi
         P.dbg_n0 = n0;
         P.dbg_n1 = n1;
     }
-    if (!debug && use_gemv(op, M, K, 1)) return launch_gemv(op, x, w_packed, scale, M, K, N, g, y, ws, s, L, stream);
+    if (!debug) {
+        const int sk = small_kernel(op, M, K, N, g, 1);
+        if (sk != kSmallNone) return launch_gemv(op, sk == kSmallMma, x, w_packed, scale, M, K, N, g, y, ws, s, L, stream);
+    }
     CUtensorMap map;
     if (op == W4A16_OP_MSD) {
         int8_t* xq = reinterpret_cast<int8_t*>(wsb + L.xq);

@@ -50,7 +50,7 @@ namespace w4a16 {
 constexpr int kGemvThreads = 256;
 constexpr int kGemvWarps = kGemvThreads / 32;
 constexpr int kGemvRound = 8;                        // 16-byte loads per thread per round
-constexpr int kGemvRecWords = 28;                    // MSD record: 24 digit words, 3 sums, 1 pad
+constexpr int kGemvRecWords = 28;                    // MSD record: 24 digit words, 3 sums, A_max
 constexpr int kGemvMaxMK = 32768;                    // M * K bound of the shared-memory operand
 
 struct GemvParams {
@@ -59,7 +59,6 @@ struct GemvParams {
     const __half* scale;      // [G][N]
     __half* y;                // [M][N]
     const uint32_t* rec;      // MSD: [K/32][M][28] digit records
-    const float* amax;        // MSD: [M][G]
     int M, K, N, g, G;
     int kchunks;              // ceil(K / 128)
     int npieces;              // K / 32
@@ -73,9 +72,9 @@ struct GemvCfg {
     static constexpr int kRed = kGemvWarps * MR * 32 * 4;   // cross-warp sum buffer
     __host__ __device__ static constexpr int operand_bytes(int M, int K)
     {
-        // MSD: the digit records and A_max; DEQUANT: x as fp16 and one fp32
+        // MSD: the digit records; DEQUANT: x as fp16 and one fp32
         // bias correction per (32-K piece, row)
-        return kIsMsd ? (K / 32) * M * kGemvRecWords * 4 + M * (K / 32) * 4 : M * K * 2 + (K / 32) * M * 4;
+        return kIsMsd ? (K / 32) * M * kGemvRecWords * 4 : M * K * 2 + (K / 32) * M * 4;
     }
     __host__ __device__ static constexpr int smem_bytes(int M, int K)
     {
@@ -139,10 +138,11 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p)
 // packed word j, low (h = 0: K offsets 8j + {0, 4, 1, 5}) or high (h = 1:
 // 8j + {2, 6, 3, 7}) nibbles -- the byte order of q & 0x0F0F0F0F and
 // (q >> 4) & 0x0F0F0F0F for a packed word q; words 24..26 hold -8 * (sum of
-// the piece's digits of plane i).  rec: [K/32][M][28]; amax: [M][G].
+// the piece's digits of plane i) and word 27 the A_max of the piece's group
+// (fp32 bits).  rec: [K/32][M][28].
 template <int NSUB>
 __global__ void __launch_bounds__(256) gemv_expand_kernel(const __half* __restrict__ x, int M, int K, int g,
-                                                          uint32_t* __restrict__ rec, float* __restrict__ amax)
+                                                          uint32_t* __restrict__ rec)
 {
     // the matmul that reads the records may launch now and stream its
     // weights; x may come from the previous kernel, and the previous matmul
@@ -152,7 +152,6 @@ __global__ void __launch_bounds__(256) gemv_expand_kernel(const __half* __restri
     const int lane = threadIdx.x & 31;
     const int span = NSUB * kKC;
     const int nspans = (K + span - 1) / span;
-    const int G = K / g;
     const long long wg = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) >> 5;
     if (wg >= static_cast<long long>(M) * nspans) return;
     const int m = static_cast<int>(wg / nspans), sp = static_cast<int>(wg % nspans);
@@ -177,15 +176,11 @@ __global__ void __launch_bounds__(256) gemv_expand_kernel(const __half* __restri
         for (int e = 0; e < 4; ++e) am = fmaxf(am, fabsf(v[s][e]));
     }
     // A_max of each group: g >= 128 spans the warp's whole span; g < 128
-    // covers g/4 consecutive lanes
+    // covers g/4 consecutive lanes; every lane ends with its group's value
     const int lanes_per_group = g >= kKC ? 32 : g / 4;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1)
         if (o < lanes_per_group) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-    if ((lane % lanes_per_group) == 0) {
-        const int k0 = sp * span + 4 * lane;
-        if (k0 < K) amax[static_cast<size_t>(m) * G + k0 / g] = am;
-    }
 
 #pragma unroll
     for (int s = 0; s < NSUB; ++s) {
@@ -232,6 +227,8 @@ __global__ void __launch_bounds__(256) gemv_expand_kernel(const __half* __restri
                 if ((lane & 7) == 0) r[24 + i] = static_cast<uint32_t>(-8 * t);
             }
         }
+        // a piece lies inside one group (g % 32 == 0)
+        if (k0 < K && (lane & 7) == 0) r[27] = __float_as_uint(am);
     }
 }
 
@@ -246,7 +243,6 @@ __global__ void __launch_bounds__(kGemvThreads, 2) gemv_kernel(const __grid_cons
     uint8_t* operand = smem + C::kRed;
     const int rec_words = P.npieces * P.M * kGemvRecWords;
     const uint32_t* rec_s = reinterpret_cast<const uint32_t*>(operand);
-    const float* amax_s = reinterpret_cast<const float*>(operand + rec_words * 4);
     const __half* xs = reinterpret_cast<const __half*>(operand);
     float* xcorr = reinterpret_cast<float*>(operand + P.M * P.K * 2);   // DEQUANT: [K/32][M]
 
@@ -354,7 +350,9 @@ __global__ void __launch_bounds__(kGemvThreads, 2) gemv_kernel(const __grid_cons
                         const float v = fmaf(static_cast<float>(yacc[m][2]), kC3,
                                              fmaf(static_cast<float>(yacc[m][1]), kC2,
                                                   static_cast<float>(yacc[m][0]) * kC1));
-                        acc[m] = fmaf(v, amax_s[m * P.G + grp] * scl, acc[m]);
+                        // word 27 of a record is the A_max of its group
+                        const float amx = __uint_as_float(rec_s[(static_cast<size_t>(p) * M + m) * kGemvRecWords + 27]);
+                        acc[m] = fmaf(v, amx * scl, acc[m]);
                         yacc[m][0] = yacc[m][1] = yacc[m][2] = 0;
                     }
                     ++grp;
@@ -428,8 +426,6 @@ __global__ void __launch_bounds__(kGemvThreads, 2) gemv_kernel(const __grid_cons
         const uint4* src = reinterpret_cast<const uint4*>(P.rec);
         uint4* dst = reinterpret_cast<uint4*>(operand);
         for (int v = tid; v < rec_words / 4; v += kGemvThreads) dst[v] = src[v];
-        float* am = reinterpret_cast<float*>(operand + rec_words * 4);
-        for (int v = tid; v < M * P.G; v += kGemvThreads) am[v] = P.amax[v];
     } else {
         const uint4* src = reinterpret_cast<const uint4*>(P.x);
         uint4* dst = reinterpret_cast<uint4*>(operand);

@@ -1,0 +1,390 @@
+// w4a16_gemv_mma.cuh -- the decode kernel for small batches on the warp-level
+// tensor-core instructions (mma.sync), both variants.
+//
+// Operator: y = x . (antiquant_scale (.) W), "WeightQuantBatchMatmulExperiment
+// 算子深度解析" (bjdmk.com.cn/news/4847346), section 4.1 (MSD, steps 9-11)
+// and the plain dequant definition.  At a handful of tokens the matmul is a
+// weight stream; what limits a CUDA-core dot product is the instruction count
+// per weight, and the 5th-generation tcgen05 MMA, with only 16 tokens of N,
+// costs far more to issue than the tile takes to compute.  The warp-level
+// MMA takes its operands from registers, so each weight word goes from the
+// load straight into an MMA fragment:
+//
+//  * B operand = the weights: one m16n8 MMA covers 8 output columns (an
+//    "8-column block").  Lane (g, t) = (lane / 4, lane % 4) loads column g's
+//    16-byte cell of piece 4q + t of a "quad" q (four 32-K pieces, 128 K;
+//    the packed layout of repack_kernel: a cell is the 32 K values of one
+//    column), and MMA j of the quad takes word j of every lane's cell, so one
+//    quad of one block is four MMAs (MSD) or eight (dequant, K = 16 each).
+//    The MMA sums over its K slots in any order, so mixing four pieces in one
+//    MMA is exact as long as they share a group: groups are whole quads
+//    (g % 128 == 0).
+//  * MSD (m16n8k32, s8 x u8 -> s32): a word's bytes q & 0x0F0F0F0F and
+//    (q >> 4) & 0x0F0F0F0F are the weights' u = w + 8 at K offsets
+//    {0,4,1,5} / {2,6,3,7} of the word -- the fragment's two registers.  The
+//    A rows are (digit plane i, token m), row i*M + m; lane (r, t)'s A
+//    registers are words 2j, 2j+1 of plane i of piece 4q + t's digit record,
+//    which gemv_expand_kernel writes in exactly this byte order.  Y_i = D -
+//    8 * (sum of the quad's digits), exact in int32; per group the combine
+//    (equations 9-11) Y_i * c_i * A_max * scale is added to an fp32 sum per
+//    (row, column); the three planes of a token are added at the end.
+//  * DEQUANT (m16n8k16, f16 -> f32): a word unpacks to four fp16 pairs of the
+//    exact weights (K offsets (0,1), (2,3), (4,5), (6,7)); the A rows are the
+//    tokens and lane (m, t)'s A registers for word j are x[m][8j .. 8j+7] of
+//    piece 4q + t, in natural order.  The fp32 sum of a group is multiplied
+//    by its scale.
+//
+// Work split: CTA c takes the 8-column blocks [c*B/P, (c+1)*B/P); warp w
+// takes an even share of the quads of every block (a group may be cut: its
+// running sum is closed at the group's end and at the warp's last quad); the
+// warps' fp32 sums meet in shared memory and are added in warp order.  A
+// round is one quad of four blocks (32 columns): for each of the quad's
+// four pieces the warp copies the 32 columns' cells -- 512 contiguous bytes
+// of the packed layout, lane l taking column l -- with cp.async into its
+// ring in shared memory, at an XOR-swizzled slot so that the fragment reads
+// (lane (g, t) takes the cell of column g of piece 4q + t) are free of bank
+// conflicts.  Two rounds are in flight per warp, the first two issued before
+// the kernel waits for the previous grid (programmatic dependent launch), so
+// the weight stream of a call overlaps the tail of the previous one.  The
+// weights hold no registers in flight, so 16 warps of at most 64 registers
+// keep enough loads outstanding (the memory system wants many warps with a
+// few loads each) and leave room for the next call's CTA on the same SM.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include <cstdint>
+#include <type_traits>
+
+#include "sm100_ptx.cuh"
+#include "w4a16_gemv.cuh"
+#include "w4a16_kernels.cuh"
+
+namespace w4a16 {
+
+constexpr int kMgWarps = 16;
+constexpr int kMgThreads = kMgWarps * 32;
+constexpr int kMgCB = 4;     // 8-column blocks per round (one cell per lane per piece)
+constexpr int kMgDepth = 2;  // rounds in flight per warp
+constexpr int kMgRing = kMgDepth * 4 * 512 + kMgDepth * kMgCB * 16;   // weight cells + scales, per warp
+
+template <int VAR, int MR>
+struct MgCfg {
+    static constexpr bool kIsMsd = VAR == kMsd;
+    static constexpr int kRows = kIsMsd ? 3 * MR : MR;   // A / D rows in use
+    static_assert(kRows <= 8, "rows must fit the lower half of the m16 tile");
+    static constexpr int kRed = kMgWarps * kMgCB * 8 * 8 * 4;   // [warp][block][row][column] fp32
+    // the most quads (and 32-K pieces) one warp takes
+    __host__ __device__ static constexpr int qpw(int npieces) { return (npieces / 4 + kMgWarps - 1) / kMgWarps; }
+    __host__ __device__ static constexpr int ppw(int npieces) { return 4 * qpw(npieces); }
+    // one warp's operand: MSD the digit records of its pieces [ppw][M][28
+    // words]; DEQUANT its slice of x [M][ppw * 32] fp16
+    __host__ __device__ static constexpr int operand_bytes(int M, int npieces)
+    {
+        return kIsMsd ? ppw(npieces) * M * kGemvRecWords * 4 : ppw(npieces) * M * 64;
+    }
+    __host__ __device__ static constexpr int warp_stride(int M, int npieces, int ppg)
+    {
+        return (void)ppg, kMgRing + operand_bytes(M, npieces);
+    }
+    __host__ __device__ static constexpr int smem_bytes(int M, int npieces, int ppg)
+    {
+        return kRed + kMgWarps * warp_stride(M, npieces, ppg);
+    }
+};
+
+__device__ __forceinline__ uint32_t ldg_stream32(const void* p)
+{
+    uint32_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+// all but the N most recent groups of this thread's copies are complete
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// D[0..1] += A . B for the rows < 8 of an m16n8k32 tile (rows 8..15 of A are
+// zero): A signed bytes, B unsigned bytes, int32 accumulation
+__device__ __forceinline__ void mma_s8u8(int (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1)
+{
+    [[maybe_unused]] int z0, z1;
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(z0), "=r"(z1)
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "r"(d[0]), "r"(d[1]), "r"(0), "r"(0));
+    (void)z0;
+    (void)z1;
+}
+
+// D[0..1] += A . B for the rows < 8 of an m16n8k16 tile, fp16 in, fp32 sums
+__device__ __forceinline__ void mma_f16(float (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1)
+{
+    [[maybe_unused]] float z0, z1;
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(z0), "=f"(z1)
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(d[0]), "f"(d[1]), "f"(0.f), "f"(0.f));
+    (void)z0;
+    (void)z1;
+}
+
+// Eight packed weights -> four fp16 pairs of the exact signed values, K
+// offsets (0,1), (2,3), (4,5), (6,7): 0x6400 | u is 1024 + u and 0x6400 |
+// (u << 4) is 1024 + 16u in binary16 (u = w + 8), so w = (1024 + u) - 1032 =
+// (1024 + 16u) / 16 - 72, each exact.
+__device__ __forceinline__ void unpack_exact_f16(uint32_t q, uint32_t (&p)[4])
+{
+    const uint32_t q8 = q >> 8;
+    const __half2 b1032 = __half2half2(__ushort_as_half(0x6408u));   // 1032
+    const __half2 s16 = __half2half2(__ushort_as_half(0x2C00u));     // 1/16
+    const __half2 b72 = __half2half2(__ushort_as_half(0xD480u));     // -72
+    const uint32_t r0 = (q & 0x000F000Fu) | 0x64006400u;
+    const uint32_t r1 = (q & 0x00F000F0u) | 0x64006400u;
+    const uint32_t r2 = (q8 & 0x000F000Fu) | 0x64006400u;
+    const uint32_t r3 = (q8 & 0x00F000F0u) | 0x64006400u;
+    const __half2 w0 = __hsub2(*reinterpret_cast<const __half2*>(&r0), b1032);
+    const __half2 w1 = __hfma2(*reinterpret_cast<const __half2*>(&r1), s16, b72);
+    const __half2 w2 = __hsub2(*reinterpret_cast<const __half2*>(&r2), b1032);
+    const __half2 w3 = __hfma2(*reinterpret_cast<const __half2*>(&r3), s16, b72);
+    p[0] = *reinterpret_cast<const uint32_t*>(&w0);
+    p[1] = *reinterpret_cast<const uint32_t*>(&w1);
+    p[2] = *reinterpret_cast<const uint32_t*>(&w2);
+    p[3] = *reinterpret_cast<const uint32_t*>(&w3);
+}
+
+template <int VAR, int MR>
+__global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_constant__ GemvParams P)
+{
+    using C = MgCfg<VAR, MR>;
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gl = lane >> 2, tl = lane & 3;   // fragment row / column group of this lane
+    const int M = P.M, K = P.K;
+    const int ppg = P.g / 32, qpg = ppg / 4;   // pieces and quads per group
+    const int ppw = C::ppw(P.npieces);
+    float* red = reinterpret_cast<float*>(smem);   // [warp][block][row][column]
+    uint8_t* wreg = smem + C::kRed + warp * C::warp_stride(M, P.npieces, ppg);
+    uint8_t* ring = wreg;                                               // [depth][piece][32 cells], swizzled
+    uint8_t* sring = wreg + kMgDepth * 4 * 512;                         // [depth][block] 8 fp16 scales
+    const uint8_t* opnd = wreg + kMgRing;
+    const uint32_t* rec_w = reinterpret_cast<const uint32_t*>(opnd);    // MSD: [ppw][M][28]
+    const __half* xw = reinterpret_cast<const __half*>(opnd);           // DEQUANT: [M][ppw * 32]
+
+    const int b0 = static_cast<int>((static_cast<long long>(blockIdx.x) * P.nblk) / P.ctas);
+    const int b1 = static_cast<int>((static_cast<long long>(blockIdx.x + 1) * P.nblk) / P.ctas);
+    const int nq = P.npieces / 4;
+    const int qw0 = (warp * nq) / kMgWarps, qw1 = ((warp + 1) * nq) / kMgWarps;
+    const int pw0 = 4 * qw0, pw1 = 4 * qw1;
+    const int rpb = C::qpw(P.npieces);                  // rounds per block-group (same for every warp)
+    const int nbg = (b1 - b0 + kMgCB - 1) / kMgCB;
+    const int nitems = nbg * rpb;
+
+    // this lane's A row: MSD (plane, token) = (gl / M, gl % M); DEQUANT token gl
+    const bool row_ok = gl < (C::kIsMsd ? 3 * M : M);
+    const int row_m = C::kIsMsd ? gl % M : gl;
+    const int row_plane = C::kIsMsd ? gl / M : 0;
+    const float row_c = row_plane == 0 ? kC1 : (row_plane == 1 ? kC2 : kC3);
+
+    // the next kernel in the stream may start its own weight stream now
+    griddep_launch_dependents();
+
+    // round (bg, rr) -> ring slot `slot`: quad q = qw0 + rr of the 32
+    // columns of block-group bg; lane l copies column l's cell of each of the
+    // quad's pieces j to cell slot l ^ 2j of piece row j, lanes 0..3 the 8
+    // scales of block `lane` for the quad's group.  One commit group per
+    // round, empty or not.
+    auto load = [&](int slot, int bg, int rr) {
+        const int q = qw0 + rr;
+        const int c = (b0 + bg * kMgCB) * 8 + lane;   // this lane's column
+        if (bg < nbg && q < qw1) {
+            if (c < b1 * 8) {
+                const uint8_t* src = P.w + (static_cast<size_t>(c >> 7) * P.kchunks + q) * kWStage + (c & 127) * 16;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    cp_async16(smem_addr(ring + (slot * 4 + j) * 512 + ((lane ^ (2 * j)) * 16)), src + j * 2048);
+            }
+            const int b = b0 + bg * kMgCB + lane;
+            if (lane < kMgCB && b < b1)
+                cp_async16(smem_addr(sring + (slot * kMgCB + lane) * 16),
+                           P.scale + static_cast<size_t>(q / qpg) * P.N + b * 8);
+        }
+        cp_async_commit();
+    };
+
+    using Acc = typename std::conditional<C::kIsMsd, int, float>::type;
+    Acc d[kMgCB][2];        // the open group's running MMA sums
+    float acc[kMgCB][2];    // closed groups, scaled
+#pragma unroll
+    for (int k = 0; k < kMgCB; ++k) {
+        d[k][0] = d[k][1] = Acc(0);
+        acc[k][0] = acc[k][1] = 0.f;
+    }
+    int corr = 0;           // MSD: -8 * (digit sum) of the open group's quads, this lane's row
+    int gpos = 0;           // quads of the open group done
+    const int qpos0 = qw0 % qpg;
+
+    auto compute = [&](int slot, int bg, int rr) {
+        const int bb = b0 + bg * kMgCB;
+        const int nbk = min(kMgCB, b1 - bb);
+        if (rr == 0) gpos = qpos0;
+        const int q = qw0 + rr;
+        if (q < qw1) {
+            const bool closes = ++gpos == qpg || q + 1 == qw1;
+            if (gpos == qpg) gpos = 0;
+            uint4 cell[kMgCB];
+#pragma unroll
+            for (int k = 0; k < kMgCB; ++k)
+                cell[k] = *reinterpret_cast<const uint4*>(ring + (slot * 4 + tl) * 512 + (((8 * k + gl) ^ (2 * tl)) * 16));
+            const __half* sg = reinterpret_cast<const __half*>(sring + slot * kMgCB * 16) + 2 * tl;
+            if constexpr (C::kIsMsd) {
+                // lane (row, tl) reads the record of piece 4q + tl
+                const uint32_t* r = rec_w + ((4 * rr + tl) * M + row_m) * kGemvRecWords;
+                int c = row_ok ? static_cast<int>(r[24 + row_plane]) : 0;
+                c += __shfl_xor_sync(0xffffffffu, c, 1);
+                c += __shfl_xor_sync(0xffffffffu, c, 2);
+                corr += c;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint2 a = make_uint2(0u, 0u);
+                    if (row_ok) a = *reinterpret_cast<const uint2*>(r + row_plane * 8 + 2 * j);
+#pragma unroll
+                    for (int k = 0; k < kMgCB; ++k) {
+                        if (k >= nbk) break;
+                        const uint32_t w = j == 0 ? cell[k].x : (j == 1 ? cell[k].y : (j == 2 ? cell[k].z : cell[k].w));
+                        mma_s8u8(d[k], a.x, a.y, w & 0x0F0F0F0Fu, (w >> 4) & 0x0F0F0F0Fu);
+                    }
+                }
+                if (closes) {
+                    // word 27 of a record is the A_max of its group
+                    const float alpha = row_ok ? row_c * __uint_as_float(r[27]) : 0.f;
+#pragma unroll
+                    for (int k = 0; k < kMgCB; ++k) {
+                        if (k >= nbk) break;
+                        const float2 s = __half22float2(*reinterpret_cast<const __half2*>(sg + k * 8));
+                        // exact int32 -> fp32: |Y| < 2^22
+                        const float y0 = __int_as_float(d[k][0] + corr + 0x4B400000) - 12582912.f;
+                        const float y1 = __int_as_float(d[k][1] + corr + 0x4B400000) - 12582912.f;
+                        acc[k][0] = fmaf(y0, alpha * s.x, acc[k][0]);
+                        acc[k][1] = fmaf(y1, alpha * s.y, acc[k][1]);
+                        d[k][0] = d[k][1] = 0;
+                    }
+                    corr = 0;
+                }
+            } else {
+                const __half* xr = xw + row_m * ppw * 32 + (4 * rr + tl) * 32;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint4 xa = make_uint4(0u, 0u, 0u, 0u);
+                    if (row_ok) xa = *reinterpret_cast<const uint4*>(xr + 8 * j);
+#pragma unroll
+                    for (int k = 0; k < kMgCB; ++k) {
+                        if (k >= nbk) break;
+                        const uint32_t w = j == 0 ? cell[k].x : (j == 1 ? cell[k].y : (j == 2 ? cell[k].z : cell[k].w));
+                        uint32_t wp[4];
+                        unpack_exact_f16(w, wp);
+                        mma_f16(d[k], xa.x, xa.y, wp[0], wp[1]);
+                        mma_f16(d[k], xa.z, xa.w, wp[2], wp[3]);
+                    }
+                }
+                if (closes) {
+#pragma unroll
+                    for (int k = 0; k < kMgCB; ++k) {
+                        if (k >= nbk) break;
+                        const float2 s = __half22float2(*reinterpret_cast<const __half2*>(sg + k * 8));
+                        acc[k][0] = fmaf(d[k][0], s.x, acc[k][0]);
+                        acc[k][1] = fmaf(d[k][1], s.y, acc[k][1]);
+                        d[k][0] = d[k][1] = 0.f;
+                    }
+                }
+            }
+        }
+        // after the block-group's last round: add the warps' sums in warp
+        // order (and, for MSD, the three digit planes of each token), write y
+        if (rr == rpb - 1) {
+            if (gl < C::kRows) {
+#pragma unroll
+                for (int k = 0; k < kMgCB; ++k) {
+                    float* r = red + ((warp * kMgCB + k) * 8 + gl) * 8 + 2 * tl;
+                    r[0] = acc[k][0];
+                    r[1] = acc[k][1];
+                }
+            }
+            __syncthreads();
+            // thread (k, m, col) = (tid / (8M), (tid / 8) % M, tid % 8)
+            const int k = tid / (8 * M), m = (tid >> 3) - k * M, col = tid & 7;
+            if (k < nbk) {
+                const float* r = red + (k * 8) * 8 + col;
+                float s = 0.f;
+#pragma unroll
+                for (int w = 0; w < kMgWarps; ++w) {
+                    const float* rw = r + w * kMgCB * 64;
+                    if constexpr (C::kIsMsd)
+                        s += (rw[m * 8] + rw[(M + m) * 8]) + rw[(2 * M + m) * 8];
+                    else
+                        s += rw[m * 8];
+                }
+                P.y[static_cast<size_t>(m) * P.N + (bb + k) * 8 + col] = __float2half_rn(s);
+            }
+            if (bg + 1 < nbg) __syncthreads();
+#pragma unroll
+            for (int k2 = 0; k2 < kMgCB; ++k2) acc[k2][0] = acc[k2][1] = 0.f;
+        }
+    };
+
+    // rounds 0 .. depth-1 before the wait
+    int lbg = 0, lrr = 0;   // next round to load
+#pragma unroll
+    for (int s = 0; s < kMgDepth; ++s) {
+        load(s, lbg, lrr);
+        if (++lrr == rpb) {
+            lrr = 0;
+            ++lbg;
+        }
+    }
+
+    // x and the MSD records (and whatever wrote them) are valid once the
+    // previous grid is done; each warp copies only its own pieces' operand
+    griddep_wait();
+    const int npw = pw1 - pw0;
+    if constexpr (C::kIsMsd) {
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(P.rec + static_cast<size_t>(pw0) * M * kGemvRecWords);
+        const int nv = npw * M * (kGemvRecWords / 4);
+        for (int v = lane; v < nv; v += 32) cp_async16(smem_addr(opnd + v * 16), src + v * 16);
+    } else {
+        // row m's slice: npw * 4 vectors of 16 bytes
+        for (int m = 0; m < M; ++m)
+            for (int e = lane; e < npw * 4; e += 32)
+                cp_async16(smem_addr(opnd + (m * ppw * 4 + e) * 16), P.x + static_cast<size_t>(m) * K + pw0 * 32 + e * 8);
+    }
+    cp_async_commit();
+    cp_async_wait_all();
+    __syncwarp();
+
+    int cbg = 0, crr = 0;   // next round to compute
+    for (int i = 0; i < nitems; ++i) {
+        const int slot = i % kMgDepth;
+        compute(slot, cbg, crr);
+        if (++crr == rpb) {
+            crr = 0;
+            ++cbg;
+        }
+        // the slot is free again: refill it, then wait for the next round
+        __syncwarp();
+        load(slot, lbg, lrr);
+        if (++lrr == rpb) {
+            lrr = 0;
+            ++lbg;
+        }
+        cp_async_wait<kMgDepth - 1>();
+        __syncwarp();
+    }
+}
+
+}  // namespace w4a16
