@@ -110,29 +110,22 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// D[0..1] += A . B for the rows < 8 of an m16n8k32 tile (rows 8..15 of A are
-// zero): A signed bytes, B unsigned bytes, int32 accumulation
-__device__ __forceinline__ void mma_s8u8(int (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1)
+// D += A . B on an m16n8k32 tile: A signed bytes, B unsigned bytes, int32
+// sums.  The fragments are whole register tuples (a[1] and a[3], rows 8-15,
+// stay zero), so no moves are needed around the instruction.
+__device__ __forceinline__ void mma_s8u8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
 {
-    [[maybe_unused]] int z0, z1;
-    asm volatile(
-        "mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};"
-        : "=r"(d[0]), "=r"(d[1]), "=r"(z0), "=r"(z1)
-        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "r"(d[0]), "r"(d[1]), "r"(0), "r"(0));
-    (void)z0;
-    (void)z1;
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// D[0..1] += A . B for the rows < 8 of an m16n8k16 tile, fp16 in, fp32 sums
-__device__ __forceinline__ void mma_f16(float (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1)
+// D += A . B on an m16n8k16 tile, fp16 in, fp32 sums
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
 {
-    [[maybe_unused]] float z0, z1;
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};"
-        : "=f"(d[0]), "=f"(d[1]), "=f"(z0), "=f"(z1)
-        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(d[0]), "f"(d[1]), "f"(0.f), "f"(0.f));
-    (void)z0;
-    (void)z1;
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 // Eight packed weights -> four fp16 pairs of the exact signed values, K
@@ -186,10 +179,12 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
     const int nbg = (b1 - b0 + kMgCB - 1) / kMgCB;
     const int nitems = nbg * rpb;
 
-    // this lane's A row: MSD (plane, token) = (gl / M, gl % M); DEQUANT token gl
+    // this lane's A row: MSD (plane, token) = (gl / M, gl % M); DEQUANT token
+    // gl.  A lane past the real rows reads a valid row anyway: its MMA rows
+    // are never read back.
     const bool row_ok = gl < (C::kIsMsd ? 3 * M : M);
-    const int row_m = C::kIsMsd ? gl % M : gl;
-    const int row_plane = C::kIsMsd ? gl / M : 0;
+    const int row_m = gl % M;
+    const int row_plane = C::kIsMsd ? min(gl / M, 2) : 0;
     const float row_c = row_plane == 0 ? kC1 : (row_plane == 1 ? kC2 : kC3);
 
     // the next kernel in the stream may start its own weight stream now
@@ -219,11 +214,13 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
     };
 
     using Acc = typename std::conditional<C::kIsMsd, int, float>::type;
-    Acc d[kMgCB][2];        // the open group's running MMA sums
+    Acc d[kMgCB][4];        // the open group's running MMA sums (rows 8-15 unused)
     float acc[kMgCB][2];    // closed groups, scaled
+    uint32_t af[4] = {0u, 0u, 0u, 0u};   // A fragments; [1] and [3] (rows 8-15) stay zero
+    uint32_t ag[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
     for (int k = 0; k < kMgCB; ++k) {
-        d[k][0] = d[k][1] = Acc(0);
+        d[k][0] = d[k][1] = d[k][2] = d[k][3] = Acc(0);
         acc[k][0] = acc[k][1] = 0.f;
     }
     int corr = 0;           // MSD: -8 * (digit sum) of the open group's quads, this lane's row
@@ -238,32 +235,32 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
         if (q < qw1) {
             const bool closes = ++gpos == qpg || q + 1 == qw1;
             if (gpos == qpg) gpos = 0;
-            uint4 cell[kMgCB];
-#pragma unroll
-            for (int k = 0; k < kMgCB; ++k)
-                cell[k] = *reinterpret_cast<const uint4*>(ring + (slot * 4 + tl) * 512 + (((8 * k + gl) ^ (2 * tl)) * 16));
+            // word j of this lane's cell of block k (column 8k + gl, piece 4q + tl)
+            const uint32_t* cellw = reinterpret_cast<const uint32_t*>(ring + (slot * 4 + tl) * 512);
+            auto cword = [&](int k, int j) { return cellw[((8 * k + gl) ^ (2 * tl)) * 4 + j]; };
             const __half* sg = reinterpret_cast<const __half*>(sring + slot * kMgCB * 16) + 2 * tl;
             if constexpr (C::kIsMsd) {
                 // lane (row, tl) reads the record of piece 4q + tl
                 const uint32_t* r = rec_w + ((4 * rr + tl) * M + row_m) * kGemvRecWords;
-                int c = row_ok ? static_cast<int>(r[24 + row_plane]) : 0;
+                int c = static_cast<int>(r[24 + row_plane]);
+                if (!row_ok) c = 0;
                 c += __shfl_xor_sync(0xffffffffu, c, 1);
                 c += __shfl_xor_sync(0xffffffffu, c, 2);
                 corr += c;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    uint2 a = make_uint2(0u, 0u);
-                    if (row_ok) a = *reinterpret_cast<const uint2*>(r + row_plane * 8 + 2 * j);
+                    af[0] = r[row_plane * 8 + 2 * j];
+                    af[2] = r[row_plane * 8 + 2 * j + 1];
 #pragma unroll
                     for (int k = 0; k < kMgCB; ++k) {
                         if (k >= nbk) break;
-                        const uint32_t w = j == 0 ? cell[k].x : (j == 1 ? cell[k].y : (j == 2 ? cell[k].z : cell[k].w));
-                        mma_s8u8(d[k], a.x, a.y, w & 0x0F0F0F0Fu, (w >> 4) & 0x0F0F0F0Fu);
+                        const uint32_t w = cword(k, j);
+                        mma_s8u8(d[k], af, w & 0x0F0F0F0Fu, (w >> 4) & 0x0F0F0F0Fu);
                     }
                 }
                 if (closes) {
                     // word 27 of a record is the A_max of its group
-                    const float alpha = row_ok ? row_c * __uint_as_float(r[27]) : 0.f;
+                    const float alpha = row_ok ? row_c * __uint_as_float(r[27]) : 0.f;   // rows past 3M: unused
 #pragma unroll
                     for (int k = 0; k < kMgCB; ++k) {
                         if (k >= nbk) break;
@@ -273,24 +270,26 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
                         const float y1 = __int_as_float(d[k][1] + corr + 0x4B400000) - 12582912.f;
                         acc[k][0] = fmaf(y0, alpha * s.x, acc[k][0]);
                         acc[k][1] = fmaf(y1, alpha * s.y, acc[k][1]);
-                        d[k][0] = d[k][1] = 0;
+                        d[k][0] = d[k][1] = d[k][2] = d[k][3] = 0;
                     }
                     corr = 0;
                 }
             } else {
-                const __half* xr = xw + row_m * ppw * 32 + (4 * rr + tl) * 32;
+                const uint32_t* xr = reinterpret_cast<const uint32_t*>(xw + row_m * ppw * 32 + (4 * rr + tl) * 32);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    uint4 xa = make_uint4(0u, 0u, 0u, 0u);
-                    if (row_ok) xa = *reinterpret_cast<const uint4*>(xr + 8 * j);
+                    // x[8j .. 8j+3] and x[8j+4 .. 8j+7] of this lane's piece
+                    af[0] = xr[4 * j];
+                    af[2] = xr[4 * j + 1];
+                    ag[0] = xr[4 * j + 2];
+                    ag[2] = xr[4 * j + 3];
 #pragma unroll
                     for (int k = 0; k < kMgCB; ++k) {
                         if (k >= nbk) break;
-                        const uint32_t w = j == 0 ? cell[k].x : (j == 1 ? cell[k].y : (j == 2 ? cell[k].z : cell[k].w));
                         uint32_t wp[4];
-                        unpack_exact_f16(w, wp);
-                        mma_f16(d[k], xa.x, xa.y, wp[0], wp[1]);
-                        mma_f16(d[k], xa.z, xa.w, wp[2], wp[3]);
+                        unpack_exact_f16(cword(k, j), wp);
+                        mma_f16(d[k], af, wp[0], wp[1]);
+                        mma_f16(d[k], ag, wp[2], wp[3]);
                     }
                 }
                 if (closes) {
@@ -300,7 +299,7 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
                         const float2 s = __half22float2(*reinterpret_cast<const __half2*>(sg + k * 8));
                         acc[k][0] = fmaf(d[k][0], s.x, acc[k][0]);
                         acc[k][1] = fmaf(d[k][1], s.y, acc[k][1]);
-                        d[k][0] = d[k][1] = 0.f;
+                        d[k][0] = d[k][1] = d[k][2] = d[k][3] = 0.f;
                     }
                 }
             }
