@@ -165,19 +165,23 @@ int gemv_mma_rows(int op, int M)
 int gemv_mma_smem(int op, int M, int K, int g)
 {
     const int np = K / 32, ppg = g / 32;
-    // the shared-memory size does not depend on the row template argument
-    return op == W4A16_OP_MSD ? MgCfg<kMsd, 1>::smem_bytes(M, np, ppg) : MgCfg<kDeq, 1>::smem_bytes(M, np, ppg);
+    if (op == W4A16_OP_MSD)
+        return gemv_mma_rows(op, M) == 1 ? MgCfg<kMsd, 1>::smem_bytes(M, np, ppg) : MgCfg<kMsd, 2>::smem_bytes(M, np, ppg);
+    switch (gemv_mma_rows(op, M)) {
+        case 1: return MgCfg<kDeq, 1>::smem_bytes(M, np, ppg);
+        case 2: return MgCfg<kDeq, 2>::smem_bytes(M, np, ppg);
+        case 4: return MgCfg<kDeq, 4>::smem_bytes(M, np, ppg);
+        default: return MgCfg<kDeq, 8>::smem_bytes(M, np, ppg);
+    }
 }
 
 // The kernel of a dense call with a handful of rows.  Measured on B200
 // (consecutive dependent calls, weights streamed from HBM):
-//  * dequant, g % 128 == 0, M <= 8: the warp-MMA GEMV (w4a16_gemv_mma.cuh)
-//    beats the CUDA-core GEMV and the tensor-core decode tile at every size;
-//  * MSD, M == 1, up to 16 MB of weights: the CUDA-core GEMV
-//    (w4a16_gemv.cuh) -- at this size the call is a chain of two dependent
-//    kernels and the GEMV's own arithmetic is short;
-//  * MSD, M <= 2, K >= 2N: the warp-MMA GEMV;
-//  * g < 128 and M <= 4: the CUDA-core GEMV (the tensor tile is weak there);
+//  * g % 128 == 0, M <= 8 (dequant) or M <= 2 (MSD): the warp-MMA GEMV
+//    (w4a16_gemv_mma.cuh) beats the CUDA-core GEMV and the tensor-core
+//    decode tile at every size measured;
+//  * other g (32, 64) and M <= 4: the CUDA-core GEMV (w4a16_gemv.cuh), as the
+//    tensor tile is weak there;
 //  * everything else: the tensor-core decode tile.
 // W4A16_SMALL = tensor | cuda | mma forces one of them where it applies.
 enum SmallKernel { kSmallNone = 0, kSmallCuda = 1, kSmallMma = 2 };
@@ -205,9 +209,8 @@ int small_kernel(int op, int M, int K, int N, int g, int E)
     if (forced == kSmallNone) return kSmallNone;
     if (forced == kSmallCuda) return cuda_ok ? kSmallCuda : kSmallNone;
     if (forced == kSmallMma) return mma_ok ? kSmallMma : kSmallNone;
-    if (op == W4A16_OP_DEQUANT) return mma_ok ? kSmallMma : (cuda_ok ? kSmallCuda : kSmallNone);
-    if (cuda_ok && M == 1 && (g % 128 != 0 || static_cast<long long>(K) * N <= (32ll << 20))) return kSmallCuda;
-    if (mma_ok && K >= 2 * N) return kSmallMma;
+    (void)N;
+    if (mma_ok) return kSmallMma;
     if (cuda_ok && g % 128 != 0) return kSmallCuda;
     return kSmallNone;
 }

@@ -43,12 +43,12 @@
 // of the packed layout, lane l taking column l -- with cp.async into its
 // ring in shared memory, at an XOR-swizzled slot so that the fragment reads
 // (lane (g, t) takes the cell of column g of piece 4q + t) are free of bank
-// conflicts.  Two rounds are in flight per warp, the first two issued before
-// the kernel waits for the previous grid (programmatic dependent launch), so
-// the weight stream of a call overlaps the tail of the previous one.  The
-// weights hold no registers in flight, so 16 warps of at most 64 registers
-// keep enough loads outstanding (the memory system wants many warps with a
-// few loads each) and leave room for the next call's CTA on the same SM.
+// conflicts.  Two rounds (dequant) or four (MSD) are in flight per warp, the
+// first ones issued before the kernel waits for the previous grid
+// (programmatic dependent launch), so the weight stream of a call overlaps
+// the tail of the previous one.  The weights hold no registers in flight, so 16 warps of
+// at most 64 registers keep enough loads outstanding (the memory system
+// wants many warps with a few loads each).
 #pragma once
 
 #include <cuda_fp16.h>
@@ -65,15 +65,19 @@ namespace w4a16 {
 constexpr int kMgWarps = 16;
 constexpr int kMgThreads = kMgWarps * 32;
 constexpr int kMgCB = 4;     // 8-column blocks per round (one cell per lane per piece)
-constexpr int kMgDepth = 2;  // rounds in flight per warp
-constexpr int kMgRing = kMgDepth * 4 * 512 + kMgDepth * kMgCB * 16;   // weight cells + scales, per warp
+
 
 template <int VAR, int MR>
 struct MgCfg {
     static constexpr bool kIsMsd = VAR == kMsd;
     static constexpr int kRows = kIsMsd ? 3 * MR : MR;   // A / D rows in use
+    // rounds in flight per warp: 4 deep, the CTA alone on its SM (measured:
+    // deeper rings beat keeping the next call's CTA resident, except for a
+    // dequant call that only ever follows another dequant call)
+    static constexpr int kDepth = 4;
+    static constexpr int kRing = kDepth * 4 * 512 + kDepth * kMgCB * 16;   // weight cells + scales, per warp
     static_assert(kRows <= 8, "rows must fit the lower half of the m16 tile");
-    static constexpr int kRed = kMgWarps * kMgCB * 8 * 8 * 4;   // [warp][block][row][column] fp32
+    static constexpr int kRed = kMgWarps * kMgCB * kRows * 8 * 4;   // [warp][block][row][column] fp32
     // the most quads (and 32-K pieces) one warp takes
     __host__ __device__ static constexpr int qpw(int npieces) { return (npieces / 4 + kMgWarps - 1) / kMgWarps; }
     __host__ __device__ static constexpr int ppw(int npieces) { return 4 * qpw(npieces); }
@@ -85,7 +89,7 @@ struct MgCfg {
     }
     __host__ __device__ static constexpr int warp_stride(int M, int npieces, int ppg)
     {
-        return (void)ppg, kMgRing + operand_bytes(M, npieces);
+        return (void)ppg, kRing + operand_bytes(M, npieces);
     }
     __host__ __device__ static constexpr int smem_bytes(int M, int npieces, int ppg)
     {
@@ -165,8 +169,8 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
     float* red = reinterpret_cast<float*>(smem);   // [warp][block][row][column]
     uint8_t* wreg = smem + C::kRed + warp * C::warp_stride(M, P.npieces, ppg);
     uint8_t* ring = wreg;                                               // [depth][piece][32 cells], swizzled
-    uint8_t* sring = wreg + kMgDepth * 4 * 512;                         // [depth][block] 8 fp16 scales
-    const uint8_t* opnd = wreg + kMgRing;
+    uint8_t* sring = wreg + C::kDepth * 4 * 512;                         // [depth][block] 8 fp16 scales
+    const uint8_t* opnd = wreg + C::kRing;
     const uint32_t* rec_w = reinterpret_cast<const uint32_t*>(opnd);    // MSD: [ppw][M][28]
     const __half* xw = reinterpret_cast<const __half*>(opnd);           // DEQUANT: [M][ppw * 32]
 
@@ -310,7 +314,7 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
             if (gl < C::kRows) {
 #pragma unroll
                 for (int k = 0; k < kMgCB; ++k) {
-                    float* r = red + ((warp * kMgCB + k) * 8 + gl) * 8 + 2 * tl;
+                    float* r = red + ((warp * kMgCB + k) * C::kRows + gl) * 8 + 2 * tl;
                     r[0] = acc[k][0];
                     r[1] = acc[k][1];
                 }
@@ -319,11 +323,11 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
             // thread (k, m, col) = (tid / (8M), (tid / 8) % M, tid % 8)
             const int k = tid / (8 * M), m = (tid >> 3) - k * M, col = tid & 7;
             if (k < nbk) {
-                const float* r = red + (k * 8) * 8 + col;
+                const float* r = red + (k * C::kRows) * 8 + col;
                 float s = 0.f;
 #pragma unroll
                 for (int w = 0; w < kMgWarps; ++w) {
-                    const float* rw = r + w * kMgCB * 64;
+                    const float* rw = r + w * kMgCB * C::kRows * 8;
                     if constexpr (C::kIsMsd)
                         s += (rw[m * 8] + rw[(M + m) * 8]) + rw[(2 * M + m) * 8];
                     else
@@ -340,7 +344,7 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
     // rounds 0 .. depth-1 before the wait
     int lbg = 0, lrr = 0;   // next round to load
 #pragma unroll
-    for (int s = 0; s < kMgDepth; ++s) {
+    for (int s = 0; s < C::kDepth; ++s) {
         load(s, lbg, lrr);
         if (++lrr == rpb) {
             lrr = 0;
@@ -368,7 +372,7 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
 
     int cbg = 0, crr = 0;   // next round to compute
     for (int i = 0; i < nitems; ++i) {
-        const int slot = i % kMgDepth;
+        const int slot = i % C::kDepth;
         compute(slot, cbg, crr);
         if (++crr == rpb) {
             crr = 0;
@@ -381,7 +385,7 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
             lrr = 0;
             ++lbg;
         }
-        cp_async_wait<kMgDepth - 1>();
+        cp_async_wait<C::kDepth - 1>();
         __syncwarp();
     }
 }
