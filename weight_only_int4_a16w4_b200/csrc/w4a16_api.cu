@@ -203,13 +203,13 @@ int small_kernel(int op, int M, int K, int N, int g, int E)
 {
     if (E != 1 || M < 1) return kSmallNone;
     const bool mma_ok = g % 128 == 0 && M <= (op == W4A16_OP_MSD ? 2 : 8) &&
+                        static_cast<long long>(N / 8) * sm_count() < (1ll << 31) &&
                         gemv_mma_smem(op, M, K, g) <= kMaxSmemOptin;
     const bool cuda_ok = M <= 4 && static_cast<long long>(M) * K <= kGemvMaxMK;
     const int forced = small_override();
     if (forced == kSmallNone) return kSmallNone;
     if (forced == kSmallCuda) return cuda_ok ? kSmallCuda : kSmallNone;
     if (forced == kSmallMma) return mma_ok ? kSmallMma : kSmallNone;
-    (void)N;
     if (mma_ok) return kSmallMma;
     if (cuda_ok && g % 128 != 0) return kSmallCuda;
     return kSmallNone;

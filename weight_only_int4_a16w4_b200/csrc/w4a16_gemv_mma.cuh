@@ -174,12 +174,14 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
     const uint32_t* rec_w = reinterpret_cast<const uint32_t*>(opnd);    // MSD: [ppw][M][28]
     const __half* xw = reinterpret_cast<const __half*>(opnd);           // DEQUANT: [M][ppw * 32]
 
-    const int b0 = static_cast<int>((static_cast<long long>(blockIdx.x) * P.nblk) / P.ctas);
-    const int b1 = static_cast<int>((static_cast<long long>(blockIdx.x + 1) * P.nblk) / P.ctas);
+    // (the host keeps nblk * ctas below 2^31)
+    const int b0 = static_cast<int>((blockIdx.x * static_cast<unsigned>(P.nblk)) / static_cast<unsigned>(P.ctas));
+    const int b1 = static_cast<int>(((blockIdx.x + 1) * static_cast<unsigned>(P.nblk)) / static_cast<unsigned>(P.ctas));
     const int nq = P.npieces / 4;
     const int qw0 = (warp * nq) / kMgWarps, qw1 = ((warp + 1) * nq) / kMgWarps;
     const int pw0 = 4 * qw0, pw1 = 4 * qw1;
     const int rpb = C::qpw(P.npieces);                  // rounds per block-group (same for every warp)
+    const int gw0 = qw0 / qpg, qpos0 = qw0 - gw0 * qpg;  // the warp's first group, its quads before qw0
     const int nbg = (b1 - b0 + kMgCB - 1) / kMgCB;
     const int nitems = nbg * rpb;
 
@@ -187,8 +189,15 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
     // gl.  A lane past the real rows reads a valid row anyway: its MMA rows
     // are never read back.
     const bool row_ok = gl < (C::kIsMsd ? 3 * M : M);
-    const int row_m = gl % M;
-    const int row_plane = C::kIsMsd ? min(gl / M, 2) : 0;
+    int row_m, row_plane;
+    if constexpr (C::kIsMsd) {
+        // M is 1 or 2 here
+        row_m = M == 1 ? 0 : (gl & 1);
+        row_plane = min(M == 1 ? gl : (gl >> 1), 2);
+    } else {
+        row_m = gl < M ? gl : 0;
+        row_plane = 0;
+    }
     const float row_c = row_plane == 0 ? kC1 : (row_plane == 1 ? kC2 : kC3);
 
     // the next kernel in the stream may start its own weight stream now
@@ -199,7 +208,7 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
     // quad's pieces j to cell slot l ^ 2j of piece row j, lanes 0..3 the 8
     // scales of block `lane` for the quad's group.  One commit group per
     // round, empty or not.
-    auto load = [&](int slot, int bg, int rr) {
+    auto load = [&](int slot, int bg, int rr, int grp) {
         const int q = qw0 + rr;
         const int c = (b0 + bg * kMgCB) * 8 + lane;   // this lane's column
         if (bg < nbg && q < qw1) {
@@ -212,7 +221,7 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
             const int b = b0 + bg * kMgCB + lane;
             if (lane < kMgCB && b < b1)
                 cp_async16(smem_addr(sring + (slot * kMgCB + lane) * 16),
-                           P.scale + static_cast<size_t>(q / qpg) * P.N + b * 8);
+                           P.scale + static_cast<size_t>(grp) * P.N + b * 8);
         }
         cp_async_commit();
     };
@@ -229,7 +238,6 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
     }
     int corr = 0;           // MSD: -8 * (digit sum) of the open group's quads, this lane's row
     int gpos = 0;           // quads of the open group done
-    const int qpos0 = qw0 % qpg;
 
     auto compute = [&](int slot, int bg, int rr) {
         const int bb = b0 + bg * kMgCB;
@@ -320,9 +328,9 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
                 }
             }
             __syncthreads();
-            // thread (k, m, col) = (tid / (8M), (tid / 8) % M, tid % 8)
-            const int k = tid / (8 * M), m = (tid >> 3) - k * M, col = tid & 7;
-            if (k < nbk) {
+            // thread (k, m, col) = (tid / (8 MR), (tid / 8) % MR, tid % 8)
+            const int k = tid / (8 * MR), m = (tid >> 3) % MR, col = tid & 7;
+            if (k < nbk && m < M) {
                 const float* r = red + (k * C::kRows) * 8 + col;
                 float s = 0.f;
 #pragma unroll
@@ -341,15 +349,25 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
         }
     };
 
-    // rounds 0 .. depth-1 before the wait
-    int lbg = 0, lrr = 0;   // next round to load
-#pragma unroll
-    for (int s = 0; s < C::kDepth; ++s) {
-        load(s, lbg, lrr);
+    // rounds 0 .. depth-1 before the wait; the load cursor carries the
+    // round's block-group, quad index and the quad's group (position in it)
+    int lbg = 0, lrr = 0, lgrp = gw0, lgpos = qpos0;
+    auto advance_load = [&]() {
+        if (++lgpos == qpg) {
+            lgpos = 0;
+            ++lgrp;
+        }
         if (++lrr == rpb) {
             lrr = 0;
             ++lbg;
+            lgrp = gw0;
+            lgpos = qpos0;
         }
+    };
+#pragma unroll
+    for (int s = 0; s < C::kDepth; ++s) {
+        load(s, lbg, lrr, lgrp);
+        advance_load();
     }
 
     // x and the MSD records (and whatever wrote them) are valid once the
@@ -380,11 +398,8 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
         }
         // the slot is free again: refill it, then wait for the next round
         __syncwarp();
-        load(slot, lbg, lrr);
-        if (++lrr == rpb) {
-            lrr = 0;
-            ++lbg;
-        }
+        load(slot, lbg, lrr, lgrp);
+        advance_load();
         cp_async_wait<C::kDepth - 1>();
         __syncwarp();
     }
