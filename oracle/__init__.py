@@ -47,6 +47,8 @@ def _load():
         lib.oracle_msd_at.argtypes = [P, P, P, I, I, I, I, I, P, P, I, P]
         lib.oracle_dequant.argtypes = [P, P, P, I, I, I, I, P]
         lib.oracle_dequant_at.argtypes = [P, P, P, I, I, I, I, P, P, I, P]
+        lib.oracle_moe_align.argtypes = [P, I, I, I, P, P, P]
+        lib.oracle_moe_combine.argtypes = [P, P, P, I, I, I, P]
         lib.oracle_num_threads.restype = I
         _lib = lib
     return _lib
@@ -226,3 +228,52 @@ def grouped_at(op: str, x, wps, scales, offsets, g, rows, cols) -> np.ndarray:
         a, b = int(offsets[e]), int(offsets[e + 1])
         out[sel] = fn(x[a:b], wps[e], scales[e], g, rows[sel] - a, cols[sel])
     return out
+
+
+def moe_align(topk_ids, E):
+    """Stable grouping of the router's entries by expert (reading R8 of the C
+    file): returns offsets [E+1], sorted_token [T*topk], inv_pos [T*topk] and
+    the number of entries whose id lies outside [0, E)."""
+    ids = _c(np.asarray(topk_ids, np.int32), np.int32)
+    T, topk = ids.shape
+    offsets = np.empty(E + 1, np.int32)
+    st = np.empty(T * topk, np.int32)
+    inv = np.empty(T * topk, np.int32)
+    dropped = _load().oracle_moe_align(_ptr(ids), T, topk, E, _ptr(offsets), _ptr(st), _ptr(inv))
+    if dropped < 0:
+        raise ValueError("oracle moe_align failed")
+    return offsets, st, inv, dropped
+
+
+def moe_combine(y_sorted, inv_pos, weights):
+    """Gate-weighted un-permute (reading R9): fp16 y_sorted [rows, N] -> fp16 y [T, N]."""
+    ys = _c(np.asarray(y_sorted, np.float16), np.float16)
+    inv = _c(np.asarray(inv_pos, np.int32), np.int32)
+    w = _c(np.asarray(weights, np.float32), np.float32)
+    T, topk = w.shape
+    N = ys.shape[1]
+    y = np.empty((T, N), np.uint16)
+    _check(_load().oracle_moe_combine(_ptr(ys), _ptr(inv), _ptr(w), T, topk, N, _ptr(y)), "moe_combine")
+    return y.view(np.float16)
+
+
+def moe(op: str, x, topk_ids, weights, wps, scales, g) -> np.ndarray:
+    """The routed grouped form end to end: y [T, N] float64.
+
+    The entries are grouped by expert (moe_align), the per-expert matmul runs
+    on the gathered rows (grouped), and token t's rows are added with its
+    gate weights in binary64 (no binary16 rounding in between)."""
+    x = _c(x, np.float16)
+    w = np.asarray(weights, np.float64)
+    T, topk = w.shape
+    offsets, st, inv, _ = moe_align(topk_ids, len(wps))
+    rows = int(offsets[-1])
+    xs = x[st[:rows]] if rows else np.zeros((0, x.shape[1]), np.float16)
+    ys = grouped(op, xs, wps, scales, offsets, g)
+    y = np.zeros((T, ys.shape[1] if rows else wps[0].shape[1]), np.float64)
+    for t in range(T):
+        for j in range(topk):
+            pos = int(inv[t * topk + j])
+            if pos >= 0:
+                y[t] += w[t, j] * ys[pos]
+    return y

@@ -33,6 +33,7 @@
  *       (section 4.3: "each byte stores two int4").
  *   R7  eq. 10-11 are evaluated in binary64, groups added in increasing order,
  *       and y is rounded to binary16 (round-to-nearest-even) once at the end.
+ *   R8, R9  the routing prep of the grouped form (see oracle_moe_align).
  *
  * Build: gcc -O2 -fopenmp -ffp-contract=off -fno-fast-math -fPIC -shared
  * (binary32 arithmetic must stay IEEE single with no FMA contraction).
@@ -365,6 +366,76 @@ int oracle_dequant_at(const uint16_t* x, const uint8_t* wp, const uint16_t* scal
         y[i] = acc;
     }
     return bad ? -3 : 0;
+}
+
+/* ---------------------------------------------------------------------- */
+/* Routing prep for the grouped (per-expert) form.                          */
+/*                                                                          */
+/* The grouped matmul takes each expert's tokens as one contiguous segment  */
+/* of rows (offsets[E+1]); the mixture-of-experts scheduling of the Humming */
+/* article (aihirek.info, MoE section) and the moe_align_block_size step of */
+/* the FlagGems operator list (pwwt.cn) both start from a router's          */
+/* topk_ids [T][topk].  Reading R8: the routing prep is a stable grouping  */
+/* of the entries i = t*topk + j (token t's j-th expert) by expert id, in   */
+/* increasing i within an expert; an id outside [0, E) takes no row.  R9:   */
+/* the un-permute adds token t's rows weighted by its gate weights,         */
+/* slots in increasing j, in binary64, rounded to binary16 once.            */
+/* ---------------------------------------------------------------------- */
+
+/* offsets[e] = entries whose expert is below e; entry i of expert e gets row
+ * pos = offsets[e] + (entries of expert e before i); sorted_token[pos] = t
+ * (its token) and inv_pos[i] = pos.  Entries without an expert get
+ * inv_pos[i] = -1 and rows offsets[E] .. T*topk-1 hold -1.  Returns the
+ * number of such entries. */
+int oracle_moe_align(const int32_t* ids, int T, int topk, int E, int32_t* offsets,
+                     int32_t* sorted_token, int32_t* inv_pos)
+{
+    const int n = T * topk;
+    int64_t* fill = (int64_t*)calloc((size_t)E + 1, sizeof(int64_t));
+    if (!fill) return -1;
+    int dropped = 0;
+    for (int e = 0; e <= E; ++e) offsets[e] = 0;
+    for (int i = 0; i < n; ++i) {
+        const int e = ids[i];
+        if (e < 0 || e >= E) {
+            ++dropped;
+            continue;
+        }
+        ++offsets[e + 1];
+    }
+    for (int e = 0; e < E; ++e) offsets[e + 1] += offsets[e];
+    for (int i = 0; i < n; ++i) sorted_token[i] = -1;
+    for (int i = 0; i < n; ++i) {
+        const int e = ids[i];
+        if (e < 0 || e >= E) {
+            inv_pos[i] = -1;
+            continue;
+        }
+        const int pos = offsets[e] + (int)fill[e]++;
+        sorted_token[pos] = i / topk;
+        inv_pos[i] = pos;
+    }
+    free(fill);
+    return dropped;
+}
+
+/* y[t][n] = sum_j w[t][j] * y_sorted[inv_pos[t*topk+j]][n] (binary16 in and
+ * out, binary64 sum, slots in increasing j, entries without a row skipped). */
+int oracle_moe_combine(const uint16_t* y_sorted, const int32_t* inv_pos, const float* w, int T, int topk,
+                       int N, uint16_t* y)
+{
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t)
+        for (int n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int j = 0; j < topk; ++j) {
+                const int pos = inv_pos[t * topk + j];
+                if (pos < 0) continue;
+                acc += (double)w[t * topk + j] * oracle_half_to_double(y_sorted[(size_t)pos * N + n]);
+            }
+            y[(size_t)t * N + n] = oracle_double_to_half(acc);
+        }
+    return 0;
 }
 
 /* Threads an OpenMP parallel region will use (for the CPU-baseline report). */

@@ -302,3 +302,78 @@ def test_workload_table():
     assert (workload(2).M, workload(2).N) == (16, 14336)
     assert (workload(3).M, workload(3).N) == (4096, 4096)
     assert (workload(4).E, workload(4).M, workload(4).N) == (8, 4096, 14336)
+
+
+# ---------------------------------------------------------------- routing prep of the grouped form
+
+def _numpy_grouping(ids, E):
+    """Independent reference: numpy's stable argsort of the expert ids (ids
+    outside [0, E) sort last and take no row)."""
+    flat = ids.reshape(-1).astype(np.int64)
+    key = np.where((flat >= 0) & (flat < E), flat, E)
+    order = np.argsort(key, kind="stable")
+    valid = int(np.sum(key < E))
+    counts = np.bincount(key, minlength=E + 1)[:E]
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    sorted_token = np.full(flat.size, -1, np.int32)
+    sorted_token[:valid] = order[:valid] // ids.shape[1]
+    inv = np.full(flat.size, -1, np.int32)
+    inv[order[:valid]] = np.arange(valid)
+    return offsets, sorted_token, inv, flat.size - valid
+
+
+@pytest.mark.parametrize("T,topk,E,lo", [(1, 1, 1, 0), (37, 2, 8, -1), (256, 8, 64, 0), (500, 3, 5, -2)])
+def test_moe_align_is_a_stable_grouping(T, topk, E, lo):
+    rng = np.random.default_rng(T * 31 + topk)
+    ids = rng.integers(lo, E + 1, (T, topk)).astype(np.int32)      # includes invalid ids when lo < 0 or = E
+    got = oracle.moe_align(ids, E)
+    ref = _numpy_grouping(ids, E)
+    for a, b in zip(got[:3], ref[:3]):
+        np.testing.assert_array_equal(a, b)
+    assert got[3] == ref[3]
+
+
+def test_moe_combine_topk1_unit_weight_is_the_permutation():
+    rng = np.random.default_rng(5)
+    ids = rng.integers(0, 4, (50, 1)).astype(np.int32)
+    _, _, inv, _ = oracle.moe_align(ids, 4)
+    ys = rng.standard_normal((50, 24)).astype(np.float16)
+    y = oracle.moe_combine(ys, inv, np.ones((50, 1), np.float32))
+    np.testing.assert_array_equal(y.view(np.uint16), ys[inv].view(np.uint16))
+
+
+def test_moe_combine_is_linear_in_the_gate_weights():
+    """A one-hot weight picks one slot's row exactly; doubling every weight
+    doubles the result exactly (a power-of-two scale commutes with rounding)."""
+    rng = np.random.default_rng(6)
+    T, topk, E, N = 40, 3, 6, 16
+    ids = rng.integers(0, E, (T, topk)).astype(np.int32)
+    _, _, inv, _ = oracle.moe_align(ids, E)
+    ys = (rng.standard_normal((T * topk, N)) * 0.25).astype(np.float16)
+    for j in range(topk):
+        w = np.zeros((T, topk), np.float32)
+        w[:, j] = 1
+        np.testing.assert_array_equal(oracle.moe_combine(ys, inv, w).view(np.uint16),
+                                      ys[inv.reshape(T, topk)[:, j]].view(np.uint16))
+    w = rng.uniform(0, 1, (T, topk)).astype(np.float32)
+    a = oracle.moe_combine(ys, inv, w).astype(np.float64)
+    b = oracle.moe_combine(ys, inv, 2 * w).astype(np.float64)
+    np.testing.assert_array_equal(2 * a, b)
+
+
+def test_moe_pipeline_matches_per_token_experts():
+    """The routed pipeline equals, token by token, the gate-weighted sum of
+    the token's own experts' dequant products (no permutation involved)."""
+    rng = np.random.default_rng(7)
+    T, topk, E, K, N, g = 9, 2, 3, 64, 16, 32
+    c = make_case(T, K, N, g, seed=11, E=E)
+    ids = rng.integers(-1, E, (T, topk)).astype(np.int32)
+    w = rng.uniform(0, 1, (T, topk)).astype(np.float32)
+    got = oracle.moe("dequant", c.x, ids, w, c.wp, c.scale, g)
+    ref = np.zeros((T, N))
+    for t in range(T):
+        for j in range(topk):
+            e = ids[t, j]
+            if 0 <= e < E:
+                ref[t] += float(w[t, j]) * oracle.dequant(c.x[t:t + 1], c.wp[e], c.scale[e], g)[0]
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
