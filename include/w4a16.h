@@ -62,14 +62,15 @@ typedef enum {
     W4A16_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. g = 96)   */
     W4A16_ERR_WORKSPACE = 3,     /* workspace missing or smaller than needed  */
     W4A16_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed      */
-    W4A16_ERR_TIMEOUT = 5        /* a device wait expired (see status word)   */
+    W4A16_ERR_TIMEOUT = 5,       /* a device wait expired (see status word)   */
+    W4A16_ERR_BAD_INDEX = 6      /* a device-side index was out of range      */
 } w4a16_status;
 
 /* Operation selector for w4a16_workspace_size and w4a16_grouped_matmul. */
 enum { W4A16_OP_MSD = 0, W4A16_OP_DEQUANT = 1 };
 
 /* Bits of the device status word kept at the start of every workspace. */
-enum { W4A16_DEVICE_TIMEOUT = 1u };
+enum { W4A16_DEVICE_TIMEOUT = 1u, W4A16_DEVICE_BAD_EXPERT = 2u };
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* w4a16_status_string(w4a16_status s);
@@ -148,6 +149,58 @@ w4a16_status w4a16_grouped_matmul(int op, const void* x, const void* const* w_pa
                                   void* workspace, size_t workspace_bytes,
                                   w4a16_stream_t stream);
 
+/* ---- routing prep of the grouped form (mixture of experts) --------------
+ * A router gives, per token t, topk expert ids topk_ids[t][j] and gate
+ * weights.  The grouped matmul wants each expert's rows contiguous; the
+ * steps below group the router's entries i = t*topk + j by expert, gather x
+ * into that order, run the grouped matmul and add each token's rows back
+ * with its gate weights -- the dense/MoE scheduling of the Humming article
+ * (aihirek.info, MoE section) from the moe_align_block_size-style routing
+ * step of the FlagGems operator list (pwwt.cn).  Plain reading taken: a
+ * stable grouping (increasing i within an expert); an id outside [0, E)
+ * takes no row, contributes nothing and sets W4A16_DEVICE_BAD_EXPERT. */
+
+/* Stable grouping of the entries by expert.
+ *   topk_ids      device int32 [T][topk]
+ *   offsets       device int32 [E+1]: offsets[e] = entries whose expert < e
+ *   sorted_token  device int32 [T*topk]: row r of the sorted order holds
+ *                 the token of its entry; rows >= offsets[E] hold -1
+ *   inv_pos       device int32 [T*topk]: the row of entry i, or -1
+ *   workspace     device, >= 256 bytes, status word at its start (zeroed
+ *                 by the caller before first use)
+ * 1 <= E <= 64, topk >= 1, T >= 0, T*topk < 2^31. */
+w4a16_status w4a16_moe_align(const int32_t* topk_ids, int T, int topk, int E, int32_t* offsets,
+                             int32_t* sorted_token, int32_t* inv_pos, void* workspace,
+                             size_t workspace_bytes, w4a16_stream_t stream);
+
+/* x_sorted[r] = x[sorted_token[r]] (fp16 rows of K values; zero where
+ * sorted_token[r] < 0).  x, x_sorted 16-byte aligned, K % 8 == 0. */
+w4a16_status w4a16_moe_gather(const void* x, const int32_t* sorted_token, int rows, int K,
+                              void* x_sorted, w4a16_stream_t stream);
+
+/* y[t] = sum_j topk_weights[t][j] * y_sorted[inv_pos[t*topk+j]] (fp16 rows of
+ * N values, fp32 sums in increasing j, entries with inv_pos < 0 skipped,
+ * fp16 out).  y_sorted, y 16-byte aligned, N % 8 == 0. */
+w4a16_status w4a16_moe_combine(const void* y_sorted, const int32_t* inv_pos,
+                               const float* topk_weights, int T, int topk, int N, void* y,
+                               w4a16_stream_t stream);
+
+/* Workspace of w4a16_moe_matmul: the grouped matmul's own workspace for
+ * T*topk rows, then offsets, sorted_token, inv_pos, the gathered x and the
+ * per-row y. */
+w4a16_status w4a16_moe_workspace_size(int op, int T, int topk, int K, int N, int group_size,
+                                      int E, size_t* bytes);
+
+/* The routed grouped form end to end: align, gather, grouped matmul,
+ * combine, on one stream, no host synchronisation.  x fp16 [T][K], y fp16
+ * [T][N]; w_packed / scale as w4a16_grouped_matmul; topk_ids, topk_weights
+ * device [T][topk]. */
+w4a16_status w4a16_moe_matmul(int op, const void* x, const int32_t* topk_ids,
+                              const float* topk_weights, const void* const* w_packed,
+                              const void* const* scale, int E, int T, int topk, int K, int N,
+                              int group_size, void* y, void* workspace, size_t workspace_bytes,
+                              w4a16_stream_t stream);
+
 /* Debug window into MSD equation 9: the exact int32 Y1, Y2, Y3 per group
  * for rows m0..m1-1 and columns n0..n1-1, as accumulated by the tensor
  * cores, plus A_max.
@@ -190,9 +243,11 @@ w4a16_status w4a16_msd_matmul_noalloc(const void* x, const void* w_packed, const
                                       w4a16_stream_t stream);
 
 /* Copy the device status word at the start of `workspace` into *status
- * (0 = no device error; W4A16_DEVICE_TIMEOUT bit = a bounded wait expired).
+ * (0 = no device error; W4A16_DEVICE_TIMEOUT bit = a bounded wait expired;
+ * W4A16_DEVICE_BAD_EXPERT bit = a router id outside [0, E)).
  * SYNCHRONISES `stream`.  Returns W4A16_ERR_TIMEOUT when the timeout bit is
- * set, W4A16_OK otherwise. */
+ * set, else W4A16_ERR_BAD_INDEX when the bad-expert bit is set, else
+ * W4A16_OK. */
 w4a16_status w4a16_read_status(const void* workspace, w4a16_stream_t stream,
                                uint32_t* status);
 

@@ -113,3 +113,32 @@ def test_repack_rejects(lib):
         lib.w4a16_repack(fake, 256, 250, fake, stream=0)     # N % 8
     with pytest.raises(lib.W4A16Error):
         lib.w4a16_repack(fake, 256, 256, fake + 8, stream=0)  # misaligned output
+
+
+def test_moe_entry_points_reject_before_launch(lib):
+    fake = 1 << 40
+    cases = [
+        (lambda: lib.w4a16_moe_align(fake, 4, 2, 0, fake, fake, fake, fake, 1 << 20, stream=0), 1),    # E = 0
+        (lambda: lib.w4a16_moe_align(fake, 4, 2, 65, fake, fake, fake, fake, 1 << 20, stream=0), 1),   # E > 64
+        (lambda: lib.w4a16_moe_align(fake, 4, 0, 8, fake, fake, fake, fake, 1 << 20, stream=0), 1),    # topk = 0
+        (lambda: lib.w4a16_moe_align(fake, 4, 2, 8, fake, fake, fake, fake, 16, stream=0), 3),         # workspace
+        (lambda: lib.w4a16_moe_gather(fake, fake, 4, 12, fake, stream=0), 1),                          # K % 8
+        (lambda: lib.w4a16_moe_gather(fake + 8, fake, 4, 16, fake, stream=0), 1),                      # misaligned x
+        (lambda: lib.w4a16_moe_combine(fake, fake, fake, 4, 2, 20, fake, stream=0), 1),                # N % 8
+        (lambda: lib.w4a16_moe_combine(fake, None, fake, 4, 2, 16, fake, stream=0), 1),                # null inv_pos
+        (lambda: lib.w4a16_moe_workspace_size(0, 4, 2, 576, 256, 96, 8), 2),                           # g = 96
+    ]
+    for fn, code in cases:
+        with pytest.raises(lib.W4A16Error) as e:
+            fn()
+        assert e.value.code == code
+    # empty inputs are no-ops that touch nothing
+    lib.w4a16_moe_gather(None, None, 0, 16, None, stream=0)
+    lib.w4a16_moe_combine(None, None, None, 0, 2, 16, None, stream=0)
+
+
+def test_moe_workspace_holds_every_intermediate(lib):
+    T, topk, K, N, g, E = 100, 2, 512, 264, 64, 8
+    total = lib.w4a16_moe_workspace_size(1, T, topk, K, N, g, E)
+    grouped = lib.w4a16_workspace_size(1, T * topk, K, N, g, E)
+    assert total >= grouped + (E + 1) * 4 + 2 * T * topk * 4 + T * topk * (K + N) * 2

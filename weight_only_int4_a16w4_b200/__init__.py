@@ -25,9 +25,11 @@ _lib = ctypes.CDLL(LIB_PATH)
 OP_MSD = 0
 OP_DEQUANT = 1
 DEVICE_TIMEOUT = 1
+DEVICE_BAD_EXPERT = 2
 
 _STATUS_NAMES = {0: "W4A16_OK", 1: "W4A16_ERR_INVALID_ARG", 2: "W4A16_ERR_UNSUPPORTED",
-                 3: "W4A16_ERR_WORKSPACE", 4: "W4A16_ERR_CUDA", 5: "W4A16_ERR_TIMEOUT"}
+                 3: "W4A16_ERR_WORKSPACE", 4: "W4A16_ERR_CUDA", 5: "W4A16_ERR_TIMEOUT",
+                 6: "W4A16_ERR_BAD_INDEX"}
 
 
 class W4A16Error(RuntimeError):
@@ -57,6 +59,16 @@ _lib.w4a16_msd_debug_yint.restype = _I
 _lib.w4a16_msd_debug_yint.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]
 _lib.w4a16_msd_matmul_noalloc.restype = _I
 _lib.w4a16_msd_matmul_noalloc.argtypes = [_P, _P, _P, _I, _I, _I, _I, _P, _P]
+_lib.w4a16_moe_align.restype = _I
+_lib.w4a16_moe_align.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]
+_lib.w4a16_moe_gather.restype = _I
+_lib.w4a16_moe_gather.argtypes = [_P, _P, _I, _I, _P, _P]
+_lib.w4a16_moe_combine.restype = _I
+_lib.w4a16_moe_combine.argtypes = [_P, _P, _P, _I, _I, _I, _P, _P]
+_lib.w4a16_moe_workspace_size.restype = _I
+_lib.w4a16_moe_workspace_size.argtypes = [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)]
+_lib.w4a16_moe_matmul.restype = _I
+_lib.w4a16_moe_matmul.argtypes = [_I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]
 _lib.w4a16_read_status.restype = _I
 _lib.w4a16_read_status.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_uint32)]
 _lib.w4a16_set_wait_timeout_ns.restype = None
@@ -140,6 +152,40 @@ def w4a16_msd_debug_yint(x, w_packed, M, K, N, group_size, m0, m1, n0, n1, yint,
            "w4a16_msd_debug_yint")
 
 
+def w4a16_moe_align(topk_ids, T, topk, E, offsets, sorted_token, inv_pos, workspace, workspace_bytes=None,
+                    stream=None):
+    wb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check(_lib.w4a16_moe_align(_ptr(topk_ids), T, topk, E, _ptr(offsets), _ptr(sorted_token), _ptr(inv_pos),
+                                _ptr(workspace), wb, _stream(stream)), "w4a16_moe_align")
+
+
+def w4a16_moe_gather(x, sorted_token, rows, K, x_sorted, stream=None):
+    _check(_lib.w4a16_moe_gather(_ptr(x), _ptr(sorted_token), rows, K, _ptr(x_sorted), _stream(stream)),
+           "w4a16_moe_gather")
+
+
+def w4a16_moe_combine(y_sorted, inv_pos, topk_weights, T, topk, N, y, stream=None):
+    _check(_lib.w4a16_moe_combine(_ptr(y_sorted), _ptr(inv_pos), _ptr(topk_weights), T, topk, N, _ptr(y),
+                                  _stream(stream)), "w4a16_moe_combine")
+
+
+def w4a16_moe_workspace_size(op, T, topk, K, N, group_size, E) -> int:
+    out = _SZ(0)
+    _check(_lib.w4a16_moe_workspace_size(op, T, topk, K, N, group_size, E, ctypes.byref(out)),
+           "w4a16_moe_workspace_size")
+    return int(out.value)
+
+
+def w4a16_moe_matmul(op, x, topk_ids, topk_weights, w_packed_list, scale_list, E, T, topk, K, N, group_size, y,
+                     workspace, workspace_bytes=None, stream=None):
+    wb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    wp = (ctypes.c_void_p * E)(*[_ptr(t) for t in w_packed_list])
+    sp = (ctypes.c_void_p * E)(*[_ptr(t) for t in scale_list])
+    _check(_lib.w4a16_moe_matmul(op, _ptr(x), _ptr(topk_ids), _ptr(topk_weights), ctypes.cast(wp, _P),
+                                 ctypes.cast(sp, _P), E, T, topk, K, N, group_size, _ptr(y), _ptr(workspace), wb,
+                                 _stream(stream)), "w4a16_moe_matmul")
+
+
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -154,7 +200,7 @@ def w4a16_read_status(workspace, stream=None) -> int:
     """Device status word of a workspace (synchronises the stream)."""
     out = ctypes.c_uint32(0)
     code = _lib.w4a16_read_status(_ptr(workspace), _stream(stream), ctypes.byref(out))
-    if code not in (0, 5):
+    if code not in (0, 5, 6):
         _check(code, "w4a16_read_status")
     return int(out.value)
 

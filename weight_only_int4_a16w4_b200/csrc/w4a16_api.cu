@@ -16,6 +16,7 @@
 #include "w4a16_gemv.cuh"
 #include "w4a16_gemv_mma.cuh"
 #include "w4a16_kernels.cuh"
+#include "w4a16_moe.cuh"
 
 using namespace w4a16;
 
@@ -625,6 +626,7 @@ const char* w4a16_status_string(w4a16_status s)
         case W4A16_ERR_WORKSPACE: return "workspace missing or too small";
         case W4A16_ERR_CUDA: return "CUDA error";
         case W4A16_ERR_TIMEOUT: return "device wait timed out";
+        case W4A16_ERR_BAD_INDEX: return "device-side index out of range";
     }
     return "unknown status";
 }
@@ -732,6 +734,111 @@ w4a16_status w4a16_grouped_matmul(int op, const void* x, const void* const* w_pa
     return launch_for(op, s.TT, map, P, grid, cs);
 }
 
+w4a16_status w4a16_moe_align(const int32_t* topk_ids, int T, int topk, int E, int32_t* offsets,
+                             int32_t* sorted_token, int32_t* inv_pos, void* workspace, size_t workspace_bytes,
+                             w4a16_stream_t stream)
+{
+    if (T < 0 || topk < 1 || E < 1 || E > kMoeMaxExperts) return W4A16_ERR_INVALID_ARG;
+    if (static_cast<long long>(T) * topk >= (1ll << 31)) return W4A16_ERR_INVALID_ARG;
+    if (!offsets || !workspace) return W4A16_ERR_INVALID_ARG;
+    if (workspace_bytes < kHeaderBytes) return W4A16_ERR_WORKSPACE;
+    if (T > 0 && (!topk_ids || !sorted_token || !inv_pos)) return W4A16_ERR_INVALID_ARG;
+    moe_align_kernel<<<1, kMoeAlignThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        topk_ids, T * topk, topk, E, offsets, sorted_token, inv_pos, static_cast<uint32_t*>(workspace));
+    return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+}
+
+w4a16_status w4a16_moe_gather(const void* x, const int32_t* sorted_token, int rows, int K, void* x_sorted,
+                              w4a16_stream_t stream)
+{
+    if (rows < 0 || K <= 0 || K % 8) return W4A16_ERR_INVALID_ARG;
+    if (rows == 0) return W4A16_OK;
+    if (!x || !sorted_token || !x_sorted || !aligned16(x) || !aligned16(x_sorted)) return W4A16_ERR_INVALID_ARG;
+    moe_gather_kernel<<<cdiv(rows, 8), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4*>(x), sorted_token, rows, K / 8, static_cast<uint4*>(x_sorted));
+    return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+}
+
+w4a16_status w4a16_moe_combine(const void* y_sorted, const int32_t* inv_pos, const float* topk_weights, int T,
+                               int topk, int N, void* y, w4a16_stream_t stream)
+{
+    if (T < 0 || topk < 1 || N <= 0 || N % 8) return W4A16_ERR_INVALID_ARG;
+    if (static_cast<long long>(T) * topk >= (1ll << 31)) return W4A16_ERR_INVALID_ARG;
+    if (T == 0) return W4A16_OK;
+    if (!y_sorted || !inv_pos || !topk_weights || !y || !aligned16(y_sorted) || !aligned16(y))
+        return W4A16_ERR_INVALID_ARG;
+    moe_combine_kernel<<<cdiv(T, 8), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        static_cast<const __half*>(y_sorted), inv_pos, topk_weights, T, topk, N, static_cast<__half*>(y));
+    return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+}
+
+namespace {
+struct MoeLayout {
+    size_t grouped = 0, offsets = 0, sorted = 0, inv = 0, xs = 0, ys = 0, total = 0;
+};
+
+w4a16_status moe_layout(int op, int T, int topk, int K, int N, int g, int E, MoeLayout* L)
+{
+    if (T < 0 || topk < 1) return W4A16_ERR_INVALID_ARG;
+    const long long rows = static_cast<long long>(T) * topk;
+    if (rows >= (1ll << 31)) return W4A16_ERR_INVALID_ARG;
+    size_t gws = 0;
+    const w4a16_status st = w4a16_workspace_size(op, static_cast<int>(rows), K, N, g, E, &gws);
+    if (st != W4A16_OK) return st;
+    size_t off = align256(gws);
+    L->grouped = gws;
+    L->offsets = off;
+    off += align256(static_cast<size_t>(E + 1) * 4);
+    L->sorted = off;
+    off += align256(static_cast<size_t>(rows) * 4);
+    L->inv = off;
+    off += align256(static_cast<size_t>(rows) * 4);
+    L->xs = off;
+    off += align256(static_cast<size_t>(rows) * K * 2);
+    L->ys = off;
+    off += align256(static_cast<size_t>(rows) * N * 2);
+    L->total = off;
+    return W4A16_OK;
+}
+}  // namespace
+
+w4a16_status w4a16_moe_workspace_size(int op, int T, int topk, int K, int N, int group_size, int E, size_t* bytes)
+{
+    if (!bytes) return W4A16_ERR_INVALID_ARG;
+    MoeLayout L;
+    const w4a16_status st = moe_layout(op, T, topk, K, N, group_size, E, &L);
+    if (st == W4A16_OK) *bytes = L.total;
+    return st;
+}
+
+w4a16_status w4a16_moe_matmul(int op, const void* x, const int32_t* topk_ids, const float* topk_weights,
+                              const void* const* w_packed, const void* const* scale, int E, int T, int topk, int K,
+                              int N, int group_size, void* y, void* workspace, size_t workspace_bytes,
+                              w4a16_stream_t stream)
+{
+    MoeLayout L;
+    w4a16_status st = moe_layout(op, T, topk, K, N, group_size, E, &L);
+    if (st != W4A16_OK) return st;
+    if (T == 0) return W4A16_OK;
+    if (!x || !topk_ids || !topk_weights || !y || !workspace) return W4A16_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(workspace)) return W4A16_ERR_INVALID_ARG;
+    if (workspace_bytes < L.total) return W4A16_ERR_WORKSPACE;
+    uint8_t* wsb = static_cast<uint8_t*>(workspace);
+    int32_t* offsets = reinterpret_cast<int32_t*>(wsb + L.offsets);
+    int32_t* sorted = reinterpret_cast<int32_t*>(wsb + L.sorted);
+    int32_t* inv = reinterpret_cast<int32_t*>(wsb + L.inv);
+    const int rows = T * topk;
+    // the grouped matmul's workspace comes first, so the status word at the
+    // start of `workspace` is shared by every step
+    if ((st = w4a16_moe_align(topk_ids, T, topk, E, offsets, sorted, inv, workspace, L.grouped, stream)) != W4A16_OK)
+        return st;
+    if ((st = w4a16_moe_gather(x, sorted, rows, K, wsb + L.xs, stream)) != W4A16_OK) return st;
+    if ((st = w4a16_grouped_matmul(op, wsb + L.xs, w_packed, scale, offsets, E, rows, K, N, group_size, wsb + L.ys,
+                                   workspace, L.grouped, stream)) != W4A16_OK)
+        return st;
+    return w4a16_moe_combine(wsb + L.ys, inv, topk_weights, T, topk, N, y, stream);
+}
+
 w4a16_status w4a16_msd_matmul_noalloc(const void* x, const void* w_packed, const void* scale, int M, int K, int N,
                                       int group_size, void* y, w4a16_stream_t stream)
 {
@@ -755,7 +862,8 @@ w4a16_status w4a16_read_status(const void* workspace, w4a16_stream_t stream, uin
     if (cudaMemcpyAsync(status, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost, cs) != cudaSuccess)
         return W4A16_ERR_CUDA;
     if (cudaStreamSynchronize(cs) != cudaSuccess) return W4A16_ERR_CUDA;
-    return (*status & W4A16_DEVICE_TIMEOUT) ? W4A16_ERR_TIMEOUT : W4A16_OK;
+    if (*status & W4A16_DEVICE_TIMEOUT) return W4A16_ERR_TIMEOUT;
+    return (*status & W4A16_DEVICE_BAD_EXPERT) ? W4A16_ERR_BAD_INDEX : W4A16_OK;
 }
 
 void w4a16_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns); }

@@ -1,0 +1,162 @@
+// w4a16_moe.cuh -- routing prep of the grouped (mixture-of-experts) form.
+//
+// The grouped matmul takes each expert's tokens as one contiguous segment of
+// rows (offsets[E+1]); a router hands over topk_ids [T][topk] (token t's
+// j-th expert) and gate weights.  The mixture-of-experts scheduling of the
+// Humming article (aihirek.info, MoE section) and the moe_align_block_size
+// step of the FlagGems operator list (pwwt.cn) start from exactly that.
+// Three kernels:
+//
+//  * moe_align_kernel: a stable grouping of the entries i = t*topk + j by
+//    expert (increasing i within an expert): offsets, the token of every
+//    sorted row and every entry's row.  One CTA of 32 warps; warp w owns a
+//    contiguous run of entries, counts its experts with __match_any_sync (one
+//    leader per expert per 32 entries), the per-(warp, expert) counts are
+//    turned into row bases by a scan over (expert, warp), and a second walk
+//    places each entry at base + (its rank among equal experts before it in
+//    the same 32).  The result is unique, so it is compared bit for bit.  An
+//    id outside [0, E) takes no row and sets W4A16_DEVICE_BAD_EXPERT.
+//  * moe_gather_kernel: x rows into sorted order (a warp per row, 16-byte
+//    loads); rows without an entry are zero.
+//  * moe_combine_kernel: y[t] = sum_j w[t][j] * y_sorted[row of (t, j)], fp32
+//    sums in increasing j, fp16 out (a warp per token, 8 columns per lane
+//    per step).
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include <cstdint>
+
+namespace w4a16 {
+
+constexpr int kMoeAlignThreads = 1024;
+constexpr int kMoeAlignWarps = kMoeAlignThreads / 32;
+constexpr int kMoeMaxExperts = 64;
+constexpr uint32_t kDeviceBadExpert = 2u;   // status bit (W4A16_DEVICE_BAD_EXPERT)
+
+__global__ void __launch_bounds__(kMoeAlignThreads) moe_align_kernel(const int32_t* __restrict__ ids, int n, int topk,
+                                                                     int E, int32_t* __restrict__ offsets,
+                                                                     int32_t* __restrict__ sorted_token,
+                                                                     int32_t* __restrict__ inv_pos,
+                                                                     uint32_t* __restrict__ status)
+{
+    __shared__ int cnt[kMoeAlignWarps][kMoeMaxExperts];   // counts, then running row bases
+    __shared__ int off_s[kMoeMaxExperts + 1];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c0 = static_cast<int>((static_cast<long long>(warp) * n) / kMoeAlignWarps);
+    const int c1 = static_cast<int>((static_cast<long long>(warp + 1) * n) / kMoeAlignWarps);
+    for (int e = lane; e < kMoeMaxExperts; e += 32) cnt[warp][e] = 0;
+    __syncwarp();
+
+    auto key_of = [&](int i) {
+        if (i >= c1) return -1;
+        const int e = ids[i];
+        return (e >= 0 && e < E) ? e : -1;
+    };
+
+    // counts per (warp, expert)
+    for (int base = c0; base < c1; base += 32) {
+        const int key = key_of(base + lane);
+        const unsigned peers = __match_any_sync(0xffffffffu, key);
+        if (key >= 0 && lane == __ffs(peers) - 1) cnt[warp][key] += __popc(peers);
+        __syncwarp();
+    }
+    __syncthreads();
+
+    // offsets[e] = entries of the experts below e; then cnt[w][e] = the row
+    // of warp w's first entry of expert e
+    if (tid < E) {
+        int tot = 0;
+        for (int w = 0; w < kMoeAlignWarps; ++w) tot += cnt[w][tid];
+        off_s[tid + 1] = tot;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        off_s[0] = 0;
+        for (int e = 0; e < E; ++e) off_s[e + 1] += off_s[e];
+    }
+    __syncthreads();
+    if (tid <= E) offsets[tid] = off_s[tid];
+    if (tid < E) {
+        int run = off_s[tid];
+        for (int w = 0; w < kMoeAlignWarps; ++w) {
+            const int c = cnt[w][tid];
+            cnt[w][tid] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+
+    // place every entry
+    const unsigned below = (1u << lane) - 1u;
+    for (int base = c0; base < c1; base += 32) {
+        const int i = base + lane;
+        const int key = key_of(i);
+        const unsigned peers = __match_any_sync(0xffffffffu, key);
+        if (key >= 0) {
+            const int pos = cnt[warp][key] + __popc(peers & below);
+            sorted_token[pos] = i / topk;
+            inv_pos[i] = pos;
+        } else if (i < c1) {
+            inv_pos[i] = -1;
+            atomicOr(status, kDeviceBadExpert);
+        }
+        __syncwarp();
+        if (key >= 0 && lane == __ffs(peers) - 1) cnt[warp][key] += __popc(peers);
+        __syncwarp();
+    }
+    // rows no entry took
+    for (int p = off_s[E] + tid; p < n; p += kMoeAlignThreads) sorted_token[p] = -1;
+}
+
+// x_sorted[r] = x[sorted_token[r]] (zero where sorted_token[r] < 0); kv =
+// K / 8 16-byte vectors per row; a warp per row.
+__global__ void __launch_bounds__(256) moe_gather_kernel(const uint4* __restrict__ x,
+                                                         const int32_t* __restrict__ sorted_token, int rows, int kv,
+                                                         uint4* __restrict__ x_sorted)
+{
+    const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const int src = sorted_token[row];
+    uint4* dst = x_sorted + static_cast<size_t>(row) * kv;
+    if (src < 0) {
+        for (int v = lane; v < kv; v += 32) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+        return;
+    }
+    const uint4* s = x + static_cast<size_t>(src) * kv;
+    for (int v = lane; v < kv; v += 32) dst[v] = s[v];
+}
+
+// y[t][c .. c+7] = sum_j w[t][j] * y_sorted[inv_pos[t*topk+j]][c .. c+7],
+// fp32 sums in increasing j (entries without a row skipped), a warp per token.
+__global__ void __launch_bounds__(256) moe_combine_kernel(const __half* __restrict__ y_sorted,
+                                                          const int32_t* __restrict__ inv_pos,
+                                                          const float* __restrict__ weights, int T, int topk, int N,
+                                                          __half* __restrict__ y)
+{
+    const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (t >= T) return;
+    for (int c = lane * 8; c < N; c += 256) {
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int j = 0; j < topk; ++j) {
+            const int pos = inv_pos[t * topk + j];
+            if (pos < 0) continue;
+            const float wj = weights[t * topk + j];
+            const uint4 v = *reinterpret_cast<const uint4*>(y_sorted + static_cast<size_t>(pos) * N + c);
+            const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float2 f = __half22float2(h[q]);
+                acc[2 * q] = fmaf(wj, f.x, acc[2 * q]);
+                acc[2 * q + 1] = fmaf(wj, f.y, acc[2 * q + 1]);
+            }
+        }
+        uint4 out;
+        __half2* o = reinterpret_cast<__half2*>(&out);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) o[q] = __floats2half2_rn(acc[2 * q], acc[2 * q + 1]);
+        *reinterpret_cast<uint4*>(y + static_cast<size_t>(t) * N + c) = out;
+    }
+}
+
+}  // namespace w4a16
