@@ -17,10 +17,10 @@
 //    the same 32).  The result is unique, so it is compared bit for bit.  An
 //    id outside [0, E) takes no row and sets W4A16_DEVICE_BAD_EXPERT.
 //  * moe_gather_kernel: x rows into sorted order (a warp per row, 16-byte
-//    loads); rows without an entry are zero.
+//    loads, four in flight per lane); rows without an entry are zero.
 //  * moe_combine_kernel: y[t] = sum_j w[t][j] * y_sorted[row of (t, j)], fp32
-//    sums in increasing j, fp16 out (a warp per token, 8 columns per lane
-//    per step).
+//    sums in increasing j, fp16 out (a warp per token, four 16-byte loads in
+//    flight per lane).
 #pragma once
 
 #include <cuda_fp16.h>
@@ -110,11 +110,13 @@ __global__ void __launch_bounds__(kMoeAlignThreads) moe_align_kernel(const int32
 }
 
 // x_sorted[r] = x[sorted_token[r]] (zero where sorted_token[r] < 0); kv =
-// K / 8 16-byte vectors per row; a warp per row.
+// K / 8 16-byte vectors per row; a warp per row, four loads in flight per
+// lane.
 __global__ void __launch_bounds__(256) moe_gather_kernel(const uint4* __restrict__ x,
                                                          const int32_t* __restrict__ sorted_token, int rows, int kv,
                                                          uint4* __restrict__ x_sorted)
 {
+    constexpr int U = 4;
     const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     if (row >= rows) return;
     const int src = sorted_token[row];
@@ -124,38 +126,65 @@ __global__ void __launch_bounds__(256) moe_gather_kernel(const uint4* __restrict
         return;
     }
     const uint4* s = x + static_cast<size_t>(src) * kv;
-    for (int v = lane; v < kv; v += 32) dst[v] = s[v];
+    for (int v0 = lane; v0 < kv; v0 += 32 * U) {
+        uint4 t[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if (v0 + 32 * u < kv) t[u] = s[v0 + 32 * u];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if (v0 + 32 * u < kv) dst[v0 + 32 * u] = t[u];
+    }
 }
 
 // y[t][c .. c+7] = sum_j w[t][j] * y_sorted[inv_pos[t*topk+j]][c .. c+7],
-// fp32 sums in increasing j (entries without a row skipped), a warp per token.
+// fp32 sums in increasing j (entries without a row skipped), a warp per
+// token; each lane keeps four 16-byte loads in flight (columns c, c + 256,
+// c + 512, c + 768).
 __global__ void __launch_bounds__(256) moe_combine_kernel(const __half* __restrict__ y_sorted,
                                                           const int32_t* __restrict__ inv_pos,
                                                           const float* __restrict__ weights, int T, int topk, int N,
                                                           __half* __restrict__ y)
 {
+    constexpr int U = 4;
     const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     if (t >= T) return;
-    for (int c = lane * 8; c < N; c += 256) {
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int c0 = lane * 8; c0 < N; c0 += 256 * U) {
+        float acc[U][8];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[u][q] = 0.f;
         for (int j = 0; j < topk; ++j) {
             const int pos = inv_pos[t * topk + j];
             if (pos < 0) continue;
             const float wj = weights[t * topk + j];
-            const uint4 v = *reinterpret_cast<const uint4*>(y_sorted + static_cast<size_t>(pos) * N + c);
-            const __half2* h = reinterpret_cast<const __half2*>(&v);
+            const __half* row = y_sorted + static_cast<size_t>(pos) * N;
+            uint4 v[U];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float2 f = __half22float2(h[q]);
-                acc[2 * q] = fmaf(wj, f.x, acc[2 * q]);
-                acc[2 * q + 1] = fmaf(wj, f.y, acc[2 * q + 1]);
+            for (int u = 0; u < U; ++u)
+                if (c0 + 256 * u < N) v[u] = *reinterpret_cast<const uint4*>(row + c0 + 256 * u);
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (c0 + 256 * u >= N) break;
+                const __half2* h = reinterpret_cast<const __half2*>(&v[u]);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float2 f = __half22float2(h[q]);
+                    acc[u][2 * q] = fmaf(wj, f.x, acc[u][2 * q]);
+                    acc[u][2 * q + 1] = fmaf(wj, f.y, acc[u][2 * q + 1]);
+                }
             }
         }
-        uint4 out;
-        __half2* o = reinterpret_cast<__half2*>(&out);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) o[q] = __floats2half2_rn(acc[2 * q], acc[2 * q + 1]);
-        *reinterpret_cast<uint4*>(y + static_cast<size_t>(t) * N + c) = out;
+        for (int u = 0; u < U; ++u) {
+            if (c0 + 256 * u >= N) break;
+            uint4 out;
+            __half2* o = reinterpret_cast<__half2*>(&out);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) o[q] = __floats2half2_rn(acc[u][2 * q], acc[u][2 * q + 1]);
+            *reinterpret_cast<uint4*>(y + static_cast<size_t>(t) * N + c0 + 256 * u) = out;
+        }
     }
 }
 
