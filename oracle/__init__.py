@@ -231,7 +231,7 @@ def grouped_at(op: str, x, wps, scales, offsets, g, rows, cols) -> np.ndarray:
 
 
 def moe_align(topk_ids, E):
-    """Stable grouping of the router's entries by expert (reading R8 of the C
+    """Stable grouping of the router's entries by expert (reading R13 of the C
     file): returns offsets [E+1], sorted_token [T*topk], inv_pos [T*topk] and
     the number of entries whose id lies outside [0, E)."""
     ids = _c(np.asarray(topk_ids, np.int32), np.int32)
@@ -246,7 +246,7 @@ def moe_align(topk_ids, E):
 
 
 def moe_combine(y_sorted, inv_pos, weights):
-    """Gate-weighted un-permute (reading R9): fp16 y_sorted [rows, N] -> fp16 y [T, N]."""
+    """Gate-weighted un-permute (reading R14): fp16 y_sorted [rows, N] -> fp16 y [T, N]."""
     ys = _c(np.asarray(y_sorted, np.float16), np.float16)
     inv = _c(np.asarray(inv_pos, np.int32), np.int32)
     w = _c(np.asarray(weights, np.float32), np.float32)

@@ -33,7 +33,7 @@
  *       (section 4.3: "each byte stores two int4").
  *   R7  eq. 10-11 are evaluated in binary64, groups added in increasing order,
  *       and y is rounded to binary16 (round-to-nearest-even) once at the end.
- *   R8, R9  the routing prep of the grouped form (see oracle_moe_align).
+ *   R13, R14  the routing prep of the grouped form (see oracle_moe_align).
  *
  * Build: gcc -O2 -fopenmp -ffp-contract=off -fno-fast-math -fPIC -shared
  * (binary32 arithmetic must stay IEEE single with no FMA contraction).
@@ -375,9 +375,9 @@ int oracle_dequant_at(const uint16_t* x, const uint8_t* wp, const uint16_t* scal
 /* of rows (offsets[E+1]); the mixture-of-experts scheduling of the Humming */
 /* article (aihirek.info, MoE section) and the moe_align_block_size step of */
 /* the FlagGems operator list (pwwt.cn) both start from a router's          */
-/* topk_ids [T][topk].  Reading R8: the routing prep is a stable grouping  */
+/* topk_ids [T][topk].  Reading R13: the routing prep is a stable grouping  */
 /* of the entries i = t*topk + j (token t's j-th expert) by expert id, in   */
-/* increasing i within an expert; an id outside [0, E) takes no row.  R9:   */
+/* increasing i within an expert; an id outside [0, E) takes no row.  R14:   */
 /* the un-permute adds token t's rows weighted by its gate weights,         */
 /* slots in increasing j, in binary64, rounded to binary16 once.            */
 /* ---------------------------------------------------------------------- */
