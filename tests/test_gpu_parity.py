@@ -303,6 +303,43 @@ def test_mma_gemv_msd(cuda_lib, M, K, N, g):
                      f"mma msd {M}x{K}x{N} g{g}")
 
 
+# Decode shapes between the GEMVs' row limits and 16 rows, g % 128 == 0
+# (the tensor-core decode tile): few column tiles, K of two chunks, groups of
+# 2-4 chunks, ragged N, the full 16 rows at the decode_m16 shape (sampled).
+SK = [
+    # (M, K, N, g)
+    (9, 4096, 264, 128),
+    (16, 1024, 64, 256),
+    (5, 2560, 1032, 512),
+    (16, 512, 4104, 128),
+    (13, 256, 2048, 128),
+    (3, 3072, 776, 384),
+    (16, 4096, 14336, 128),
+]
+
+
+@pytest.mark.parametrize("M,K,N,g", SK)
+def test_decode_tile_rows_both_variants(cuda_lib, M, K, N, g):
+    w4 = cuda_lib
+    c = make_case(M, K, N, g, seed=M * 419 + K * 23 + N + g)
+    c.x[M - 1, g:2 * g] = 0              # an all-zero group
+    dev = upload(w4, c)
+    if M * N > 20000:                    # the full oracle is slow here: sample
+        rng = np.random.default_rng(M + N)
+        rows = rng.integers(0, M, 3000)
+        cols = rng.integers(0, N, 3000)
+        ym = run_dense(w4, w4.OP_MSD, c, dev)[rows, cols]
+        yd = run_dense(w4, w4.OP_DEQUANT, c, dev)[rows, cols]
+        assert_msd_close(ym, oracle.msd_at(c.x, c.wp[0], c.scale[0], g, rows, cols), "decode msd sampled")
+        ref_d = oracle.dequant_at(c.x, c.wp[0], c.scale[0], g, rows, cols)
+        assert_deq_close(yd, ref_d, "decode dequant sampled")
+        return
+    assert_msd_close(run_dense(w4, w4.OP_MSD, c, dev), oracle.msd(c.x, c.wp[0], c.scale[0], g),
+                     f"decode msd {M}x{K}x{N} g{g}")
+    assert_deq_close(run_dense(w4, w4.OP_DEQUANT, c, dev), oracle.dequant(c.x, c.wp[0], c.scale[0], g),
+                     f"decode dequant {M}x{K}x{N} g{g}")
+
+
 def test_gemv_repeat_calls_are_deterministic(cuda_lib):
     """The tile counters reset themselves and the partials are added in CTA
     order, so repeated calls on one workspace give the same bits."""
