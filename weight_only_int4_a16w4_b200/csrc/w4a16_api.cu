@@ -109,10 +109,21 @@ struct Shape {
 
 bool small_tile(int op, int M) { (void)op; return M <= 16; }
 
-int tile_tokens(int op, int M)
+// Tokens per tile.  Dequant: 256 (MMA N = 256: each MMA carries ~136 cycles
+// of tensor work, well above its issue cost -- measured 1014 vs 786 TFLOP/s
+// at M = N = K = 4096) while that still gives at least two CTAs per SM,
+// else 128.  W4A16_DEQ_TT = 128 | 256 forces one (grouped calls: T rows).
+int tile_tokens(int op, int M, int N)
 {
     if (small_tile(op, M)) return 16;
-    return op == W4A16_OP_MSD ? 64 : 128;
+    if (op == W4A16_OP_MSD) return 64;
+    static int forced = -1;
+    if (forced < 0) {
+        const char* e = std::getenv("W4A16_DEQ_TT");
+        forced = (e && *e) ? std::atoi(e) : 0;
+    }
+    if (forced == 128 || forced == 256) return forced;
+    return static_cast<long long>(cdiv(M, 256)) * cdiv(N, kBN) >= 2ll * sm_count() ? 256 : 128;
 }
 
 // Split-K factor for a decode-sized dense call: the CTAs of one column tile
@@ -133,7 +144,7 @@ int choose_splits(int tiles, int units)
 Shape dense_shape(int op, int M, int K, int N, int g)
 {
     Shape s;
-    s.TT = tile_tokens(op, M);
+    s.TT = tile_tokens(op, M, N);
     s.kchunks = cdiv(K, kKC);
     s.n_tiles = cdiv(N, kBN);
     s.t_slots = std::max(1, cdiv(M, s.TT));
@@ -146,7 +157,7 @@ Shape dense_shape(int op, int M, int K, int N, int g)
 Shape grouped_shape(int op, int T, int K, int N, int g, int E)
 {
     Shape s;
-    s.TT = tile_tokens(op, 1 << 20);
+    s.TT = tile_tokens(op, std::max(T, 17), N);   // grouped calls never use the decode tile
     s.kchunks = cdiv(K, kKC);
     s.n_tiles = cdiv(N, kBN);
     s.t_slots = std::max(1, cdiv(T, s.TT) + E);
@@ -335,6 +346,7 @@ w4a16_status launch_for(int op, int TT, const CUtensorMap& map, const GemmParams
         return launch_gemm<kMsd, 64, 4, 4, 2, 2, 1, false>(map, P, grid, s);
     }
     if (TT == 16) return launch_gemm<kDeq, 16, 4, 12, 2, 2, 4, true>(map, P, grid, s);
+    if (TT == 256) return launch_gemm<kDeq, 256, 2, 4, 2, 2, 1, false>(map, P, grid, s);
     return launch_gemm<kDeq, 128, 4, 4, 2, 1, 2, false>(map, P, grid, s);
 }
 
@@ -391,7 +403,7 @@ void base_params(GemmParams& P, int op, int M, int K, int N, int g, const Shape&
     P.unit = s.unit;
     P.E = 1;
     // the large DEQUANT tile has one accumulator per MMA issuer (two)
-    P.issuers = (op == W4A16_OP_DEQUANT && s.TT != 16) ? 2 : 1;
+    P.issuers = (op == W4A16_OP_DEQUANT && s.TT == 128) ? 2 : 1;   // the 256-token tile has one issuer
     P.status = static_cast<uint32_t*>(ws);
     P.timeout_ns = g_timeout_ns.load();
     P.write_y = 1;
