@@ -277,9 +277,9 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
                     for (int k = 0; k < kMgCB; ++k) {
                         if (k >= nbk) break;
                         const float2 s = __half22float2(*reinterpret_cast<const __half2*>(sg + k * 8));
-                        // exact int32 -> fp32: |Y| < 2^22
-                        const float y0 = __int_as_float(d[k][0] + corr + 0x4B400000) - 12582912.f;
-                        const float y1 = __int_as_float(d[k][1] + corr + 0x4B400000) - 12582912.f;
+                        // exact int32 -> fp32 (|Y| < 2^22)
+                        const float y0 = __int2float_rn(d[k][0] + corr);
+                        const float y1 = __int2float_rn(d[k][1] + corr);
                         acc[k][0] = fmaf(y0, alpha * s.x, acc[k][0]);
                         acc[k][1] = fmaf(y1, alpha * s.y, acc[k][1]);
                         d[k][0] = d[k][1] = d[k][2] = d[k][3] = 0;

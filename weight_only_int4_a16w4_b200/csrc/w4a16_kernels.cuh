@@ -400,12 +400,6 @@ __device__ __forceinline__ bool resolve_tile(const GemmParams& P, int TT, TileCo
     return false;
 }
 
-// int32 -> binary32 for the MSD accumulators: 0x4B400000 + Y, read as a
-// binary32, is exactly 12582912 + Y for |Y| < 2^22 (1.5 * 2^23 has a unit
-// last place), so one integer add and one exact subtraction convert Y
-// (|Y| <= 7 * 8 * g <= 28672) without the slower int -> float unit.
-constexpr uint32_t kAccBiasBits = 0x4B400000u;
-constexpr float kAccBias = 12582912.0f;
 // Equation 10 with 1/7.49 factored out: Y1 + Y2/14.98 + Y3/14.98^2.
 constexpr float kR2 = static_cast<float>(1.0 / 14.98);
 constexpr float kR3 = static_cast<float>(1.0 / (14.98 * 14.98));
@@ -810,12 +804,11 @@ W4A16_ROLE_UNROLL
                         tmem_ld_wait();
 #pragma unroll
                         for (int qq = 0; qq < 8; ++qq) {
-                            // exact Y_i as floats (|Y| < 2^22: the integer add puts Y in
-                            // the mantissa of 1.5 * 2^23), then equation 10 and
-                            // equation 11's running sum
-                            const float d1 = __uint_as_float(y1[qq] + kAccBiasBits) - kAccBias;
-                            const float d2 = __uint_as_float(y2[qq] + kAccBiasBits) - kAccBias;
-                            const float d3 = __uint_as_float(y3[qq] + kAccBiasBits) - kAccBias;
+                            // exact Y_i as floats (|Y| < 2^22 < 2^24), then equation 10
+                            // and equation 11's running sum
+                            const float d1 = __int2float_rn(static_cast<int>(y1[qq]));
+                            const float d2 = __int2float_rn(static_cast<int>(y2[qq]));
+                            const float d3 = __int2float_rn(static_cast<int>(y3[qq]));
                             const float v = fmaf(d3, kR3, fmaf(d2, kR2, d1));
                             acc[8 * c + qq] = fmaf(v, am[qq] * scc, acc[8 * c + qq]);
                         }
