@@ -47,6 +47,10 @@ def _load():
         lib.oracle_msd_at.argtypes = [P, P, P, I, I, I, I, I, P, P, I, P]
         lib.oracle_dequant.argtypes = [P, P, P, I, I, I, I, P]
         lib.oracle_dequant_at.argtypes = [P, P, P, I, I, I, I, P, P, I, P]
+        lib.oracle_bf16_to_double.restype = ctypes.c_double
+        lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
+        lib.oracle_bf16s_to_double.argtypes = [P, ctypes.c_int64, P]
+        lib.oracle_dequant_bf16.argtypes = [P, P, P, I, I, I, I, P]
         lib.oracle_moe_align.argtypes = [P, I, I, I, P, P, P]
         lib.oracle_moe_combine.argtypes = [P, P, P, I, I, I, P]
         lib.oracle_num_threads.restype = I
@@ -276,4 +280,25 @@ def moe(op: str, x, topk_ids, weights, wps, scales, g) -> np.ndarray:
             pos = int(inv[t * topk + j])
             if pos >= 0:
                 y[t] += w[t, j] * ys[pos]
+    return y
+
+
+def bf16_to_double(b: np.ndarray) -> np.ndarray:
+    """bfloat16 bit patterns (uint16) -> float64 values."""
+    b = _c(np.asarray(b, dtype=np.uint16), np.uint16)
+    out = np.empty(b.shape, np.float64)
+    _load().oracle_bf16s_to_double(_ptr(b), b.size, _ptr(out))
+    return out
+
+
+def dequant_bf16(x_bits, wp, scale_bits, g) -> np.ndarray:
+    """Exact y = x . (scale (.) W) in float64 with bf16 x and scale given as
+    uint16 bit patterns [M, K] / [K/g, N] (reading R15 of the C file)."""
+    x = _c(np.asarray(x_bits, np.uint16), np.uint16)
+    wp = _c(wp, np.uint8)
+    sc = _c(np.asarray(scale_bits, np.uint16), np.uint16)
+    M, K = x.shape
+    N = wp.shape[1]
+    y = np.empty((M, N), np.float64)
+    _check(_load().oracle_dequant_bf16(_ptr(x), _ptr(wp), _ptr(sc), M, K, N, g, _ptr(y)), "dequant_bf16")
     return y

@@ -34,6 +34,7 @@
  *   R7  eq. 10-11 are evaluated in binary64, groups added in increasing order,
  *       and y is rounded to binary16 (round-to-nearest-even) once at the end.
  *   R13, R14  the routing prep of the grouped form (see oracle_moe_align).
+ *   R15  bf16 activations for the dequant form (see oracle_dequant_bf16).
  *
  * Build: gcc -O2 -fopenmp -ffp-contract=off -fno-fast-math -fPIC -shared
  * (binary32 arithmetic must stay IEEE single with no FMA contraction).
@@ -366,6 +367,52 @@ int oracle_dequant_at(const uint16_t* x, const uint8_t* wp, const uint16_t* scal
         y[i] = acc;
     }
     return bad ? -3 : 0;
+}
+
+/* ---------------------------------------------------------------------- */
+/* bf16 activations for the dequant form (the INT4 + BF16 pairing of the    */
+/* Humming article, aihirek.info).  bfloat16 is the upper half of binary32: */
+/* 1 sign bit, 8 exponent bits (bias 127), 7 fraction bits.  Reading R15:   */
+/* x, scale and y are all bf16; y is the same exact binary64 definition     */
+/* x . (scale (.) W), rounded to bf16 by the caller's tolerance check.      */
+/* ---------------------------------------------------------------------- */
+
+double oracle_bf16_to_double(uint16_t b)
+{
+    const int sign = (b >> 15) & 1;
+    const int e = (b >> 7) & 0xff;
+    const int f = b & 0x7f;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -133);                /* subnormal: f * 2^-126 * 2^-7 */
+    else if (e == 0xff)
+        v = f ? NAN : INFINITY;
+    else
+        v = ldexp((double)(128 + f), e - 134);     /* (1 + f/128) * 2^(e-127) */
+    return sign ? -v : v;
+}
+
+void oracle_bf16s_to_double(const uint16_t* b, int64_t n, double* out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_bf16_to_double(b[i]);
+}
+
+int oracle_dequant_bf16(const uint16_t* x, const uint8_t* wp, const uint16_t* scale, int M, int K, int N,
+                        int g, double* y)
+{
+    if (g <= 0 || K % g) return -1;
+    for (int m = 0; m < M; ++m)
+#pragma omp parallel for schedule(static)
+        for (int n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int k = 0; k < K; ++k) {
+                const double xv = oracle_bf16_to_double(x[(size_t)m * K + k]);
+                const double s = oracle_bf16_to_double(scale[(size_t)(k / g) * N + n]);
+                acc += xv * s * (double)weight_at(wp, N, k, n);
+            }
+            y[(size_t)m * N + n] = acc;
+        }
+    return 0;
 }
 
 /* ---------------------------------------------------------------------- */

@@ -377,3 +377,49 @@ def test_moe_pipeline_matches_per_token_experts():
             if 0 <= e < E:
                 ref[t] += float(w[t, j]) * oracle.dequant(c.x[t:t + 1], c.wp[e], c.scale[e], g)[0]
     np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- bf16 activations (dequant form)
+
+def _to_bf16_bits(v):
+    """Round-to-nearest-even float32 -> bfloat16 bit patterns, done with
+    numpy integer arithmetic on the float32 bits (independent of the oracle)."""
+    b = np.asarray(v, np.float32).view(np.uint32).astype(np.uint64)
+    b = (b + 0x7FFF + ((b >> 16) & 1)) >> 16
+    return b.astype(np.uint16)
+
+
+def test_bf16_decode_matches_float32_upper_half():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    got = oracle.bf16_to_double(bits)
+    fin = np.isfinite(ref)
+    np.testing.assert_array_equal(got[fin], ref[fin])
+    assert np.all(np.isnan(got[np.isnan(ref)]))
+    assert np.array_equal(np.isinf(got), np.isinf(ref))
+
+
+def test_dequant_bf16_matches_numpy_gemm():
+    rng = np.random.default_rng(41)
+    M, K, N, g = 5, 256, 40, 64
+    c = make_case(M, K, N, g, seed=3)
+    xb = _to_bf16_bits(rng.standard_normal((M, K)))
+    sb = _to_bf16_bits(rng.uniform(-3, 3, (K // g, N)))
+    x = (xb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    s = (sb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    w = oracle.unpack_w(c.wp[0], K, N).astype(np.float64)
+    ref = x @ (np.repeat(s, g, axis=0) * w)
+    np.testing.assert_allclose(oracle.dequant_bf16(xb, c.wp[0], sb, g), ref, rtol=1e-12, atol=1e-9)
+
+
+def test_dequant_bf16_equals_fp16_oracle_on_shared_values():
+    """Values exact in both formats (small integers x, power-of-two scales)
+    give the same y through the fp16 and the bf16 oracle."""
+    rng = np.random.default_rng(43)
+    M, K, N, g = 3, 128, 24, 32
+    c = make_case(M, K, N, g, seed=4)
+    xi = rng.integers(-8, 9, (M, K)).astype(np.float32)
+    si = np.ldexp(1.0, rng.integers(-6, 2, (K // g, N))).astype(np.float32)
+    y16 = oracle.dequant(xi.astype(np.float16), c.wp[0], si.astype(np.float16), g)
+    yb = oracle.dequant_bf16(_to_bf16_bits(xi), c.wp[0], _to_bf16_bits(si), g)
+    np.testing.assert_array_equal(y16, yb)
