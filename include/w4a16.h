@@ -66,8 +66,10 @@ typedef enum {
     W4A16_ERR_BAD_INDEX = 6      /* a device-side index was out of range      */
 } w4a16_status;
 
-/* Operation selector for w4a16_workspace_size and w4a16_grouped_matmul. */
-enum { W4A16_OP_MSD = 0, W4A16_OP_DEQUANT = 1 };
+/* Operation selector for w4a16_workspace_size, w4a16_grouped_matmul and
+ * the routed (moe) entry points.  W4A16_OP_DEQUANT_BF16 is the dequant
+ * variant with bf16 x, scale and y (see w4a16_dequant_matmul_bf16). */
+enum { W4A16_OP_MSD = 0, W4A16_OP_DEQUANT = 1, W4A16_OP_DEQUANT_BF16 = 2 };
 
 /* Bits of the device status word kept at the start of every workspace. */
 enum { W4A16_DEVICE_TIMEOUT = 1u, W4A16_DEVICE_BAD_EXPERT = 2u };
@@ -81,7 +83,7 @@ const char* w4a16_status_string(w4a16_status s);
 size_t w4a16_packed_bytes(int K, int N);
 
 /* Bytes of workspace a matmul call needs.
- *   op: W4A16_OP_MSD or W4A16_OP_DEQUANT; M: rows of x (for grouped calls,
+ *   op: one of the W4A16_OP_* codes; M: rows of x (for grouped calls,
  *   the total token count T); E: 1 for the dense calls, the expert count for
  *   w4a16_grouped_matmul.  The workspace holds the device status word, the
  *   split-K partial sums and arrival counters, and (MSD) the expanded
@@ -130,16 +132,38 @@ w4a16_status w4a16_dequant_matmul(const void* x, const void* w_packed, const voi
                                   void* workspace, size_t workspace_bytes,
                                   w4a16_stream_t stream);
 
+/* Direct dequant variant with bf16 activations: the INT4 weight + BF16
+ * activation pairing of the Humming article (aihirek.info, supported
+ * formats).  bf16 holds 8 significant bits, too few for scale * w, so the
+ * weights enter the bf16 tensor cores exactly (small integers) and each
+ * group's fp32 sum is multiplied by its scale in fp32:
+ *   y[m][n] = bf16( sum_j scale[j][n] * sum_{k in group j} x[m][k] * W[k][n] )
+ * with fp32 accumulation, y rounded to bf16 (nearest even) once.
+ *   x          device bf16 [M][K]
+ *   w_packed   device, produced by w4a16_repack for (K, N)
+ *   scale      device bf16 [K/g][N]
+ *   y          device bf16 [M][N], fully overwritten
+ *   workspace  device, >= w4a16_workspace_size(W4A16_OP_DEQUANT_BF16, M, K, N, g, 1)
+ * Shape and alignment rules as for the other entry points.  M == 0 is a
+ * no-op. */
+w4a16_status w4a16_dequant_matmul_bf16(const void* x, const void* w_packed, const void* scale,
+                                       int M, int K, int N, int group_size, void* y,
+                                       void* workspace, size_t workspace_bytes,
+                                       w4a16_stream_t stream);
+
 /* Grouped-expert (MoE) form: expert e multiplies the contiguous token rows
  * offsets[e] .. offsets[e+1]-1 of x by its own weights (the dense and MoE
  * scheduling Humming describes, aihirek.info "Humming ..." article).
- *   op         W4A16_OP_MSD or W4A16_OP_DEQUANT
- *   x          device fp16 [T][K], tokens sorted by expert
+ *   op         W4A16_OP_MSD, W4A16_OP_DEQUANT or W4A16_OP_DEQUANT_BF16
+ *   x          device fp16 [T][K] (bf16 for W4A16_OP_DEQUANT_BF16), tokens
+ *              sorted by expert
  *   w_packed   host array of E device pointers (each from w4a16_repack)
- *   scale      host array of E device pointers, fp16 [K/g][N] each
+ *   scale      host array of E device pointers, fp16 [K/g][N] each (bf16
+ *              for W4A16_OP_DEQUANT_BF16)
  *   offsets    device int32 [E+1], non-decreasing, offsets[0] = 0,
  *              offsets[E] = T (empty experts allowed)
- *   y          device fp16 [T][N], fully overwritten
+ *   y          device fp16 [T][N] (bf16 for W4A16_OP_DEQUANT_BF16), fully
+ *              overwritten
  *   workspace  >= w4a16_workspace_size(op, T, K, N, g, E)
  * 1 <= E <= 64.  Offsets that break the rules above give undefined rows
  * but no out-of-bounds access: rows are clamped to [0, T). */
@@ -173,8 +197,9 @@ w4a16_status w4a16_moe_align(const int32_t* topk_ids, int T, int topk, int E, in
                              int32_t* sorted_token, int32_t* inv_pos, void* workspace,
                              size_t workspace_bytes, w4a16_stream_t stream);
 
-/* x_sorted[r] = x[sorted_token[r]] (fp16 rows of K values; zero where
- * sorted_token[r] < 0).  x, x_sorted 16-byte aligned, K % 8 == 0. */
+/* x_sorted[r] = x[sorted_token[r]] (rows of K 16-bit values, fp16 or bf16:
+ * copied as bits; zero where sorted_token[r] < 0).  x, x_sorted 16-byte
+ * aligned, K % 8 == 0. */
 w4a16_status w4a16_moe_gather(const void* x, const int32_t* sorted_token, int rows, int K,
                               void* x_sorted, w4a16_stream_t stream);
 
@@ -185,6 +210,11 @@ w4a16_status w4a16_moe_combine(const void* y_sorted, const int32_t* inv_pos,
                                const float* topk_weights, int T, int topk, int N, void* y,
                                w4a16_stream_t stream);
 
+/* w4a16_moe_combine on bf16 rows (bf16 in, fp32 sums, bf16 out). */
+w4a16_status w4a16_moe_combine_bf16(const void* y_sorted, const int32_t* inv_pos,
+                                    const float* topk_weights, int T, int topk, int N, void* y,
+                                    w4a16_stream_t stream);
+
 /* Workspace of w4a16_moe_matmul: the grouped matmul's own workspace for
  * T*topk rows, then offsets, sorted_token, inv_pos, the gathered x and the
  * per-row y. */
@@ -193,8 +223,8 @@ w4a16_status w4a16_moe_workspace_size(int op, int T, int topk, int K, int N, int
 
 /* The routed grouped form end to end: align, gather, grouped matmul,
  * combine, on one stream, no host synchronisation.  x fp16 [T][K], y fp16
- * [T][N]; w_packed / scale as w4a16_grouped_matmul; topk_ids, topk_weights
- * device [T][topk]. */
+ * [T][N] (both bf16 for W4A16_OP_DEQUANT_BF16); w_packed / scale as
+ * w4a16_grouped_matmul; topk_ids, topk_weights device [T][topk]. */
 w4a16_status w4a16_moe_matmul(int op, const void* x, const int32_t* topk_ids,
                               const float* topk_weights, const void* const* w_packed,
                               const void* const* scale, int E, int T, int topk, int K, int N,

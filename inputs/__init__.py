@@ -27,6 +27,11 @@ offsets[E+1] (exclusive prefix sums).
 
 The page's own example (section 4.3: M=1, N=12288, K=8192, g=128, x ~ U[-3,3],
 w in [-7,7], scale ~ U[-3,3]) is available as ``page_example``.
+
+bf16 activations (the dequant variant's INT4 + BF16 pairing): ``make_case``
+with ``act="bf16"`` draws the same distributions in float32 and encodes x and
+scale as bfloat16 bit patterns (uint16, round to nearest even), the format's
+definition being the upper 16 bits of a binary32.
 """
 from dataclasses import dataclass, field
 from typing import List, Optional
@@ -74,27 +79,38 @@ def pack_int4(w: np.ndarray) -> np.ndarray:
     return (u[0::2] | (u[1::2] << 4)).astype(np.uint8)
 
 
-def draw_x(rng, M, K, outliers=True) -> np.ndarray:
+def to_bf16_bits(v) -> np.ndarray:
+    """float32 values -> bfloat16 bit patterns (uint16), round to nearest even
+    on the float32 bits (finite inputs)."""
+    b = np.asarray(v, np.float32).view(np.uint32).astype(np.uint64)
+    return ((b + 0x7FFF + ((b >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def _encode(v, act):
+    return to_bf16_bits(np.asarray(v, np.float32)) if act == "bf16" else v.astype(np.float16)
+
+
+def draw_x(rng, M, K, outliers=True, act="fp16") -> np.ndarray:
     x = rng.standard_normal((M, K), dtype=np.float32)
     if outliers:
         mask = rng.random((M, K), dtype=np.float32) < 1e-3
         x = np.where(mask, x * 20.0, x)
-    return x.astype(np.float16)
+    return _encode(x, act)
 
 
 def draw_w(rng, K, N, lo=-8, hi=7) -> np.ndarray:
     return rng.integers(lo, hi + 1, size=(K, N), dtype=np.int8)
 
 
-def draw_scale(rng, G, N, lo=0.005, hi=0.02) -> np.ndarray:
-    return rng.uniform(lo, hi, size=(G, N)).astype(np.float16)
+def draw_scale(rng, G, N, lo=0.005, hi=0.02, act="fp16") -> np.ndarray:
+    return _encode(rng.uniform(lo, hi, size=(G, N)), act)
 
 
 @dataclass
 class Case:
-    x: np.ndarray                 # fp16 [M, K]
+    x: np.ndarray                 # fp16 [M, K] (bf16 cases: uint16 bit patterns)
     wp: List[np.ndarray]          # per expert: uint8 [K/2, N]
-    scale: List[np.ndarray]       # per expert: fp16 [K/g, N]
+    scale: List[np.ndarray]       # per expert: fp16 [K/g, N] (bf16 cases: uint16)
     g: int
     offsets: Optional[np.ndarray] = None   # int32 [E+1] (grouped only)
     w: List[np.ndarray] = field(default_factory=list)  # int8 [K, N] when kept
@@ -117,10 +133,11 @@ class Case:
 
 
 def make_case(M, K, N, g, seed, E=1, outliers=True, zero_group=None,
-              keep_w=False, grouped=None) -> Case:
-    """Draw one problem.  ``grouped`` (default: E > 1) adds expert offsets."""
+              keep_w=False, grouped=None, act="fp16") -> Case:
+    """Draw one problem.  ``grouped`` (default: E > 1) adds expert offsets;
+    ``act`` = "fp16" or "bf16" (x and scale as bfloat16 bit patterns)."""
     rng = np.random.Generator(np.random.PCG64(seed))
-    x = draw_x(rng, M, K, outliers)
+    x = draw_x(rng, M, K, outliers, act)
     if zero_group is not None:
         r, k0, k1 = zero_group
         x[r, k0:k1] = 0
@@ -128,7 +145,7 @@ def make_case(M, K, N, g, seed, E=1, outliers=True, zero_group=None,
     for _ in range(E):
         w = draw_w(rng, K, N)
         wps.append(pack_int4(w))
-        scales.append(draw_scale(rng, K // g, N))
+        scales.append(draw_scale(rng, K // g, N, act=act))
         if keep_w:
             ws.append(w)
     offsets = None
@@ -139,12 +156,12 @@ def make_case(M, K, N, g, seed, E=1, outliers=True, zero_group=None,
     return Case(x, wps, scales, g, offsets, ws)
 
 
-def make_workload(name_or_index, keep_w=False) -> Case:
+def make_workload(name_or_index, keep_w=False, act="fp16") -> Case:
     idx = name_or_index if isinstance(name_or_index, int) else \
         [w.name for w in WORKLOADS].index(name_or_index)
     wl = WORKLOADS[idx]
     return make_case(wl.M, wl.K, wl.N, wl.g, SEED_BASE + idx, E=wl.E,
-                     outliers=wl.outliers, zero_group=wl.zero_group, keep_w=keep_w)
+                     outliers=wl.outliers, zero_group=wl.zero_group, keep_w=keep_w, act=act)
 
 
 def page_example(seed=SEED_BASE + 100, M=1, K=8192, N=12288, g=128) -> Case:

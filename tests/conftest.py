@@ -20,3 +20,14 @@ def cuda_lib():
         pytest.skip("no CUDA device")
     import weight_only_int4_a16w4_b200 as w4
     return w4
+
+
+def build_library():
+    """Build (or refresh) the in-tree library without importing the package,
+    which would load a stale library first."""
+    import importlib.util
+    path = os.path.join(ROOT, "weight_only_int4_a16w4_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("w4a16_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()

@@ -19,8 +19,8 @@ def _declared_functions():
 
 @pytest.fixture(scope="module")
 def lib():
-    from weight_only_int4_a16w4_b200 import build
-    build.build()
+    from conftest import build_library
+    build_library()
     import weight_only_int4_a16w4_b200 as w4
     return w4
 
@@ -28,7 +28,8 @@ def lib():
 def test_header_declares_the_entry_points():
     names = _declared_functions()
     for n in ("w4a16_repack", "w4a16_msd_matmul", "w4a16_dequant_matmul", "w4a16_grouped_matmul",
-              "w4a16_msd_debug_yint", "w4a16_workspace_size", "w4a16_packed_bytes"):
+              "w4a16_msd_debug_yint", "w4a16_workspace_size", "w4a16_packed_bytes",
+              "w4a16_dequant_matmul_bf16", "w4a16_moe_combine_bf16"):
         assert n in names
 
 
@@ -54,6 +55,10 @@ def test_workspace_sizes(lib):
     assert msd - deq >= 3 * 16 * 4096 + 32 * 16 * 4
     assert lib.w4a16_workspace_size(lib.OP_DEQUANT, 0, 256, 256, 64) >= 256
     assert lib.w4a16_workspace_size(lib.OP_MSD, 4096, 4096, 14336, 128, E=8) >= 3 * 4096 * 4096
+    # the bf16 dequant variant needs what the fp16 one needs
+    for M in (1, 8, 16, 4096):
+        assert lib.w4a16_workspace_size(lib.OP_DEQUANT_BF16, M, 4096, 14336, 128) == \
+            lib.w4a16_workspace_size(lib.OP_DEQUANT, M, 4096, 14336, 128)
 
 
 @pytest.mark.parametrize("args,code", [
@@ -63,6 +68,7 @@ def test_workspace_sizes(lib):
     ((0, -1, 4096, 4096, 128), 1),      # negative M
     ((0, 16, 4096, 4096, 1024), 2),     # MSD group larger than 512
     ((7, 16, 4096, 4096, 128), 1),      # bad op
+    ((3, 16, 4096, 4096, 128), 1),      # first code past the bf16 dequant op
 ])
 def test_workspace_size_rejects(lib, args, code):
     with pytest.raises(lib.W4A16Error) as e:
@@ -72,7 +78,7 @@ def test_workspace_size_rejects(lib, args, code):
 
 def test_matmul_rejects_before_launch(lib):
     fake = 1 << 40                       # 16-byte aligned, never dereferenced
-    for fn in (lib.w4a16_msd_matmul, lib.w4a16_dequant_matmul):
+    for fn in (lib.w4a16_msd_matmul, lib.w4a16_dequant_matmul, lib.w4a16_dequant_matmul_bf16):
         with pytest.raises(lib.W4A16Error) as e:     # null x
             fn(None, fake, fake, 16, 256, 256, 64, fake, fake, 1 << 20, stream=0)
         assert e.value.code == 1
@@ -126,6 +132,7 @@ def test_moe_entry_points_reject_before_launch(lib):
         (lambda: lib.w4a16_moe_gather(fake + 8, fake, 4, 16, fake, stream=0), 1),                      # misaligned x
         (lambda: lib.w4a16_moe_combine(fake, fake, fake, 4, 2, 20, fake, stream=0), 1),                # N % 8
         (lambda: lib.w4a16_moe_combine(fake, None, fake, 4, 2, 16, fake, stream=0), 1),                # null inv_pos
+        (lambda: lib.w4a16_moe_combine_bf16(fake + 4, fake, fake, 4, 2, 16, fake, stream=0), 1),       # misaligned rows
         (lambda: lib.w4a16_moe_workspace_size(0, 4, 2, 576, 256, 96, 8), 2),                           # g = 96
     ]
     for fn, code in cases:

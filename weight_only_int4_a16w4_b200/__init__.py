@@ -17,13 +17,14 @@ LIB_PATH = os.environ.get("W4A16_LIBRARY") or os.path.join(_PKG, "libw4a16.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m weight_only_int4_a16w4_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python weight_only_int4_a16w4_b200/build.py` "
         "(nvcc, sm_100a); this package has no CPU fallback")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
 OP_MSD = 0
 OP_DEQUANT = 1
+OP_DEQUANT_BF16 = 2
 DEVICE_TIMEOUT = 1
 DEVICE_BAD_EXPERT = 2
 
@@ -50,7 +51,7 @@ _lib.w4a16_workspace_size.restype = _I
 _lib.w4a16_workspace_size.argtypes = [_I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)]
 _lib.w4a16_repack.restype = _I
 _lib.w4a16_repack.argtypes = [_P, _I, _I, _P, _P]
-for _name in ("w4a16_msd_matmul", "w4a16_dequant_matmul"):
+for _name in ("w4a16_msd_matmul", "w4a16_dequant_matmul", "w4a16_dequant_matmul_bf16"):
     getattr(_lib, _name).restype = _I
     getattr(_lib, _name).argtypes = [_P, _P, _P, _I, _I, _I, _I, _P, _P, _SZ, _P]
 _lib.w4a16_grouped_matmul.restype = _I
@@ -63,8 +64,9 @@ _lib.w4a16_moe_align.restype = _I
 _lib.w4a16_moe_align.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]
 _lib.w4a16_moe_gather.restype = _I
 _lib.w4a16_moe_gather.argtypes = [_P, _P, _I, _I, _P, _P]
-_lib.w4a16_moe_combine.restype = _I
-_lib.w4a16_moe_combine.argtypes = [_P, _P, _P, _I, _I, _I, _P, _P]
+for _name in ("w4a16_moe_combine", "w4a16_moe_combine_bf16"):
+    getattr(_lib, _name).restype = _I
+    getattr(_lib, _name).argtypes = [_P, _P, _P, _I, _I, _I, _P, _P]
 _lib.w4a16_moe_workspace_size.restype = _I
 _lib.w4a16_moe_workspace_size.argtypes = [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)]
 _lib.w4a16_moe_matmul.restype = _I
@@ -134,6 +136,13 @@ def w4a16_dequant_matmul(x, w_packed, scale, M, K, N, group_size, y, workspace, 
                                      _ptr(workspace), wb, _stream(stream)), "w4a16_dequant_matmul")
 
 
+def w4a16_dequant_matmul_bf16(x, w_packed, scale, M, K, N, group_size, y, workspace, workspace_bytes=None,
+                              stream=None):
+    wb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check(_lib.w4a16_dequant_matmul_bf16(_ptr(x), _ptr(w_packed), _ptr(scale), M, K, N, group_size, _ptr(y),
+                                          _ptr(workspace), wb, _stream(stream)), "w4a16_dequant_matmul_bf16")
+
+
 def w4a16_grouped_matmul(op, x, w_packed_list, scale_list, offsets, E, T, K, N, group_size, y, workspace,
                          workspace_bytes=None, stream=None):
     wb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
@@ -167,6 +176,11 @@ def w4a16_moe_gather(x, sorted_token, rows, K, x_sorted, stream=None):
 def w4a16_moe_combine(y_sorted, inv_pos, topk_weights, T, topk, N, y, stream=None):
     _check(_lib.w4a16_moe_combine(_ptr(y_sorted), _ptr(inv_pos), _ptr(topk_weights), T, topk, N, _ptr(y),
                                   _stream(stream)), "w4a16_moe_combine")
+
+
+def w4a16_moe_combine_bf16(y_sorted, inv_pos, topk_weights, T, topk, N, y, stream=None):
+    _check(_lib.w4a16_moe_combine_bf16(_ptr(y_sorted), _ptr(inv_pos), _ptr(topk_weights), T, topk, N, _ptr(y),
+                                       _stream(stream)), "w4a16_moe_combine_bf16")
 
 
 def w4a16_moe_workspace_size(op, T, topk, K, N, group_size, E) -> int:

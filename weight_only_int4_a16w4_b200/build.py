@@ -1,4 +1,8 @@
-"""Build libw4a16.so in-tree for sm_100a (B200) with nvcc."""
+"""Build libw4a16.so in-tree for sm_100a (B200) with nvcc.
+
+Run it as a script (``python weight_only_int4_a16w4_b200/build.py [--force]``)
+or load it by file path: importing the package loads the library, which fails
+while the library is missing or older than an entry point of the binding."""
 import os
 import subprocess
 import sys
@@ -42,3 +46,4 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+

@@ -211,6 +211,15 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int n)
            | (static_cast<uint32_t>(128 >> 4) << 24); // M / 16
 }
 
+// kind::f16 with bf16 A and B (format 1 in both type fields), f32 D
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int n)
+{
+    return (1u << 4)                                  // D = f32
+           | (1u << 7) | (1u << 10)                   // A, B = bf16
+           | (static_cast<uint32_t>(n >> 3) << 17)    // N / 8
+           | (static_cast<uint32_t>(128 >> 4) << 24); // M / 16
+}
+
 __host__ __device__ constexpr uint32_t idesc_s8_s32(int n)
 {
     return (2u << 4)                                  // D = s32

@@ -43,6 +43,8 @@ constexpr int kMaxSmemOptin = 227 * 1024;   // dynamic shared memory a CTA may o
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 int cdiv(int a, int b) { return (a + b - 1) / b; }
 
+bool op_ok(int op) { return op == W4A16_OP_MSD || op == W4A16_OP_DEQUANT || op == W4A16_OP_DEQUANT_BF16; }
+
 bool group_ok(int g)
 {
     if (g <= 0 || g % 32) return false;
@@ -96,6 +98,12 @@ bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int el
     return r == CUDA_SUCCESS;
 }
 
+// element type of the activation tiles of a dequant call
+CUtensorMapDataType act_dtype(int op)
+{
+    return op == W4A16_OP_DEQUANT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+}
+
 // ---------------------------------------------------------------- launch shapes
 
 struct Shape {
@@ -113,10 +121,13 @@ bool small_tile(int op, int M) { (void)op; return M <= 16; }
 // of tensor work, well above its issue cost -- measured 1014 vs 786 TFLOP/s
 // at M = N = K = 4096) while that still gives at least two CTAs per SM,
 // else 128.  W4A16_DEQ_TT = 128 | 256 forces one (grouped calls: T rows).
+// bf16 dequant: 128 (its per-group accumulators take two 128-column
+// buffers of Tensor Memory; 256 tokens would not fit beside the operand).
 int tile_tokens(int op, int M, int N)
 {
     if (small_tile(op, M)) return 16;
     if (op == W4A16_OP_MSD) return 64;
+    if (op == W4A16_OP_DEQUANT_BF16) return 128;
     static int forced = -1;
     if (forced < 0) {
         const char* e = std::getenv("W4A16_DEQ_TT");
@@ -193,7 +204,7 @@ int gemv_mma_smem(int op, int M, int K, int g)
 //    (w4a16_gemv_mma.cuh) beats the CUDA-core GEMV and the tensor-core
 //    decode tile at every size measured;
 //  * other g (32, 64) and M <= 4: the CUDA-core GEMV (w4a16_gemv.cuh), as the
-//    tensor tile is weak there;
+//    tensor tile is weak there (fp16 only: bf16 takes the decode tile);
 //  * everything else: the tensor-core decode tile.
 // W4A16_SMALL = tensor | cuda | mma forces one of them where it applies.
 enum SmallKernel { kSmallNone = 0, kSmallCuda = 1, kSmallMma = 2 };
@@ -217,7 +228,7 @@ int small_kernel(int op, int M, int K, int N, int g, int E)
     const bool mma_ok = g % 128 == 0 && M <= (op == W4A16_OP_MSD ? 2 : 8) &&
                         static_cast<long long>(N / 8) * sm_count() < (1ll << 31) &&
                         gemv_mma_smem(op, M, K, g) <= kMaxSmemOptin;
-    const bool cuda_ok = M <= 4 && static_cast<long long>(M) * K <= kGemvMaxMK;
+    const bool cuda_ok = op != W4A16_OP_DEQUANT_BF16 && M <= 4 && static_cast<long long>(M) * K <= kGemvMaxMK;
     const int forced = small_override();
     if (forced == kSmallNone) return kSmallNone;
     if (forced == kSmallCuda) return cuda_ok ? kSmallCuda : kSmallNone;
@@ -334,6 +345,9 @@ w4a16_status launch_gemm(const CUtensorMap& map, const GemmParams& P, dim3 grid,
 //   larger M:         MSD <64, 4, 4, 2, 2, 1>   DEQUANT <128, 4, 4, 2, 1, 2>
 //     two converter groups; MSD's per-group combine needs two epilogue
 //     groups; DEQUANT two issuers, each into its own accumulator
+//     (<256, 2, 4, 2, 2, 1> when there are enough tiles)
+//   bf16 dequant: <16, 4, 12, 2, 2, 4, scale in epilogue> and
+//     <128, 4, 4, 2, 2, 2, scale in epilogue>
 w4a16_status launch_for(int op, int TT, const CUtensorMap& map, const GemmParams& P, dim3 grid, cudaStream_t s)
 {
     if (op == W4A16_OP_MSD) {
@@ -344,6 +358,10 @@ w4a16_status launch_for(int op, int TT, const CUtensorMap& map, const GemmParams
         }
         if (TT == 16) return launch_gemm<kMsd, 16, 8, 12, 2, 2, 4, false>(map, P, grid, s);
         return launch_gemm<kMsd, 64, 4, 4, 2, 2, 1, false>(map, P, grid, s);
+    }
+    if (op == W4A16_OP_DEQUANT_BF16) {
+        if (TT == 16) return launch_gemm<kDeqBf16, 16, 4, 12, 2, 2, 4, true>(map, P, grid, s);
+        return launch_gemm<kDeqBf16, 128, 4, 4, 2, 2, 2, true>(map, P, grid, s);
     }
     if (TT == 16) return launch_gemm<kDeq, 16, 4, 12, 2, 2, 4, true>(map, P, grid, s);
     if (TT == 256) return launch_gemm<kDeq, 256, 2, 4, 2, 2, 1, false>(map, P, grid, s);
@@ -402,8 +420,11 @@ void base_params(GemmParams& P, int op, int M, int K, int N, int g, const Shape&
     P.splits = s.splits;
     P.unit = s.unit;
     P.E = 1;
-    // the large DEQUANT tile has one accumulator per MMA issuer (two)
-    P.issuers = (op == W4A16_OP_DEQUANT && s.TT == 128) ? 2 : 1;   // the 256-token tile has one issuer
+    // the large DEQUANT tile has one accumulator per MMA issuer (two); the
+    // bf16 tile two issuers when a group is one chunk (each owns one of the
+    // per-group buffers); the 256-token tile has one issuer
+    P.issuers = (op == W4A16_OP_DEQUANT && s.TT == 128) ? 2 : 1;
+    if (op == W4A16_OP_DEQUANT_BF16 && s.TT == 128) P.issuers = (g == kKC) ? 2 : 1;
     P.status = static_cast<uint32_t*>(ws);
     P.timeout_ns = g_timeout_ns.load();
     P.write_y = 1;
@@ -526,6 +547,15 @@ w4a16_status launch_gemv(int op, bool mma, const void* x, const void* w_packed, 
         if (M == 2) return launch_gemv_mr<kMsd, 2>(P, stream);
         return launch_gemv_mr<kMsd, 4>(P, stream);
     }
+    if (op == W4A16_OP_DEQUANT_BF16) {
+        if (!mma) return W4A16_ERR_UNSUPPORTED;   // small_kernel never picks the CUDA-core GEMV for bf16
+        switch (gemv_mma_rows(op, M)) {
+            case 1: return launch_gemv_mma_mr<kDeqBf16, 1>(P, stream);
+            case 2: return launch_gemv_mma_mr<kDeqBf16, 2>(P, stream);
+            case 4: return launch_gemv_mma_mr<kDeqBf16, 4>(P, stream);
+            default: return launch_gemv_mma_mr<kDeqBf16, 8>(P, stream);
+        }
+    }
     if (mma) {
         switch (gemv_mma_rows(op, M)) {
             case 1: return launch_gemv_mma_mr<kDeq, 1>(P, stream);
@@ -587,7 +617,7 @@ w4a16_status dense_matmul(int op, const void* x, const void* w_packed, const voi
         P.amax = amax;
         if (!make_map(&map, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, 3 * M, kKC, s.TT)) return W4A16_ERR_CUDA;
     } else {
-        if (!make_map(&map, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K, M, 64, s.TT)) return W4A16_ERR_CUDA;
+        if (!make_map(&map, x, act_dtype(op), 2, K, M, 64, s.TT)) return W4A16_ERR_CUDA;
     }
     // four MMA issuers on the decode tile when a group is exactly one
     // 128-deep chunk: each issuer then owns one of the per-group
@@ -652,7 +682,7 @@ size_t w4a16_packed_bytes(int K, int N)
 w4a16_status w4a16_workspace_size(int op, int M, int K, int N, int group_size, int E, size_t* bytes)
 {
     if (!bytes) return W4A16_ERR_INVALID_ARG;
-    if (op != W4A16_OP_MSD && op != W4A16_OP_DEQUANT) return W4A16_ERR_INVALID_ARG;
+    if (!op_ok(op)) return W4A16_ERR_INVALID_ARG;
     if (E < 1 || E > kMaxExperts) return W4A16_ERR_INVALID_ARG;
     w4a16_status st = check_shape(M, K, N, group_size);
     if (st != W4A16_OK) return st;
@@ -690,6 +720,14 @@ w4a16_status w4a16_dequant_matmul(const void* x, const void* w_packed, const voi
                         workspace_bytes, reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr, 0, 0, 0, 0);
 }
 
+w4a16_status w4a16_dequant_matmul_bf16(const void* x, const void* w_packed, const void* scale, int M, int K, int N,
+                                       int group_size, void* y, void* workspace, size_t workspace_bytes,
+                                       w4a16_stream_t stream)
+{
+    return dense_matmul(W4A16_OP_DEQUANT_BF16, x, w_packed, scale, M, K, N, group_size, y, workspace,
+                        workspace_bytes, reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr, 0, 0, 0, 0);
+}
+
 w4a16_status w4a16_msd_debug_yint(const void* x, const void* w_packed, int M, int K, int N, int group_size,
                                   int m0, int m1, int n0, int n1, int32_t* yint, float* amax, void* workspace,
                                   size_t workspace_bytes, w4a16_stream_t stream)
@@ -705,7 +743,7 @@ w4a16_status w4a16_grouped_matmul(int op, const void* x, const void* const* w_pa
                                   const int32_t* offsets, int E, int T, int K, int N, int group_size, void* y,
                                   void* workspace, size_t workspace_bytes, w4a16_stream_t stream)
 {
-    if (op != W4A16_OP_MSD && op != W4A16_OP_DEQUANT) return W4A16_ERR_INVALID_ARG;
+    if (!op_ok(op)) return W4A16_ERR_INVALID_ARG;
     if (E < 1 || E > kMaxExperts) return W4A16_ERR_INVALID_ARG;
     w4a16_status st = check_shape(T, K, N, group_size);
     if (st != W4A16_OK) return st;
@@ -740,7 +778,7 @@ w4a16_status w4a16_grouped_matmul(int op, const void* x, const void* const* w_pa
         P.amax = amax;
         if (!make_map(&map, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, 3 * T, kKC, s.TT)) return W4A16_ERR_CUDA;
     } else {
-        if (!make_map(&map, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K, T, 64, s.TT)) return W4A16_ERR_CUDA;
+        if (!make_map(&map, x, act_dtype(op), 2, K, T, 64, s.TT)) return W4A16_ERR_CUDA;
     }
     dim3 grid(s.n_tiles, 1, s.t_slots);
     return launch_for(op, s.TT, map, P, grid, cs);
@@ -771,17 +809,32 @@ w4a16_status w4a16_moe_gather(const void* x, const int32_t* sorted_token, int ro
     return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
 }
 
-w4a16_status w4a16_moe_combine(const void* y_sorted, const int32_t* inv_pos, const float* topk_weights, int T,
-                               int topk, int N, void* y, w4a16_stream_t stream)
+namespace {
+w4a16_status moe_combine(bool bf16, const void* y_sorted, const int32_t* inv_pos, const float* topk_weights, int T,
+                         int topk, int N, void* y, w4a16_stream_t stream)
 {
     if (T < 0 || topk < 1 || N <= 0 || N % 8) return W4A16_ERR_INVALID_ARG;
     if (static_cast<long long>(T) * topk >= (1ll << 31)) return W4A16_ERR_INVALID_ARG;
     if (T == 0) return W4A16_OK;
     if (!y_sorted || !inv_pos || !topk_weights || !y || !aligned16(y_sorted) || !aligned16(y))
         return W4A16_ERR_INVALID_ARG;
-    moe_combine_kernel<<<cdiv(T, 8), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+    auto kern = bf16 ? moe_combine_kernel<true> : moe_combine_kernel<false>;
+    kern<<<cdiv(T, 8), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
         static_cast<const __half*>(y_sorted), inv_pos, topk_weights, T, topk, N, static_cast<__half*>(y));
     return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+}
+}  // namespace
+
+w4a16_status w4a16_moe_combine(const void* y_sorted, const int32_t* inv_pos, const float* topk_weights, int T,
+                               int topk, int N, void* y, w4a16_stream_t stream)
+{
+    return moe_combine(false, y_sorted, inv_pos, topk_weights, T, topk, N, y, stream);
+}
+
+w4a16_status w4a16_moe_combine_bf16(const void* y_sorted, const int32_t* inv_pos, const float* topk_weights, int T,
+                                    int topk, int N, void* y, w4a16_stream_t stream)
+{
+    return moe_combine(true, y_sorted, inv_pos, topk_weights, T, topk, N, y, stream);
 }
 
 namespace {
@@ -848,7 +901,7 @@ w4a16_status w4a16_moe_matmul(int op, const void* x, const int32_t* topk_ids, co
     if ((st = w4a16_grouped_matmul(op, wsb + L.xs, w_packed, scale, offsets, E, rows, K, N, group_size, wsb + L.ys,
                                    workspace, L.grouped, stream)) != W4A16_OK)
         return st;
-    return w4a16_moe_combine(wsb + L.ys, inv, topk_weights, T, topk, N, y, stream);
+    return moe_combine(op == W4A16_OP_DEQUANT_BF16, wsb + L.ys, inv, topk_weights, T, topk, N, y, stream);
 }
 
 w4a16_status w4a16_msd_matmul_noalloc(const void* x, const void* w_packed, const void* scale, int M, int K, int N,

@@ -33,6 +33,8 @@
 //    tokens and lane (m, t)'s A registers for word j are x[m][8j .. 8j+7] of
 //    piece 4q + t, in natural order.  The fp32 sum of a group is multiplied
 //    by its scale.
+//  * DEQUANT with bf16 x, scale and y (m16n8k16, bf16 -> f32): the same, the
+//    weights unpacked to exact bf16 pairs (int4_to_bf162x4).
 //
 // Work split: CTA c takes the 8-column blocks [c*B/P, (c+1)*B/P); warp w
 // takes an even share of the quads of every block (a group may be cut: its
@@ -51,6 +53,7 @@
 // wants many warps with a few loads each).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include <cstdint>
@@ -70,6 +73,7 @@ constexpr int kMgCB = 4;     // 8-column blocks per round (one cell per lane per
 template <int VAR, int MR>
 struct MgCfg {
     static constexpr bool kIsMsd = VAR == kMsd;
+    static constexpr bool kBf16 = VAR == kDeqBf16;
     static constexpr int kRows = kIsMsd ? 3 * MR : MR;   // A / D rows in use
     // rounds in flight per warp: 4 deep, the CTA alone on its SM (measured:
     // deeper rings beat keeping the next call's CTA resident, except for a
@@ -130,6 +134,22 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], u
     asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// D += A . B on an m16n8k16 tile, bf16 in, fp32 sums
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// a pair of scales (fp16, or bf16 bit patterns) as floats
+template <bool BF>
+__device__ __forceinline__ float2 scale_pair(const __half* p)
+{
+    if constexpr (BF) return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+    else return __half22float2(*reinterpret_cast<const __half2*>(p));
 }
 
 // Eight packed weights -> four fp16 pairs of the exact signed values, K
@@ -299,16 +319,22 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
                     for (int k = 0; k < kMgCB; ++k) {
                         if (k >= nbk) break;
                         uint32_t wp[4];
-                        unpack_exact_f16(cword(k, j), wp);
-                        mma_f16(d[k], af, wp[0], wp[1]);
-                        mma_f16(d[k], ag, wp[2], wp[3]);
+                        if constexpr (C::kBf16) {
+                            int4_to_bf162x4(cword(k, j), wp);
+                            mma_bf16(d[k], af, wp[0], wp[1]);
+                            mma_bf16(d[k], ag, wp[2], wp[3]);
+                        } else {
+                            unpack_exact_f16(cword(k, j), wp);
+                            mma_f16(d[k], af, wp[0], wp[1]);
+                            mma_f16(d[k], ag, wp[2], wp[3]);
+                        }
                     }
                 }
                 if (closes) {
 #pragma unroll
                     for (int k = 0; k < kMgCB; ++k) {
                         if (k >= nbk) break;
-                        const float2 s = __half22float2(*reinterpret_cast<const __half2*>(sg + k * 8));
+                        const float2 s = scale_pair<C::kBf16>(sg + k * 8);
                         acc[k][0] = fmaf(d[k][0], s.x, acc[k][0]);
                         acc[k][1] = fmaf(d[k][1], s.y, acc[k][1]);
                         d[k][0] = d[k][1] = d[k][2] = d[k][3] = 0.f;
@@ -341,7 +367,7 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
                     else
                         s += rw[m * 8];
                 }
-                P.y[static_cast<size_t>(m) * P.N + (bb + k) * 8 + col] = __float2half_rn(s);
+                store_elem<C::kBf16>(P.y + static_cast<size_t>(m) * P.N + (bb + k) * 8 + col, s);
             }
             if (bg + 1 < nbg) __syncthreads();
 #pragma unroll

@@ -39,6 +39,7 @@
 #define W4A16_ROLE_UNROLL _Pragma("unroll")
 #endif
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include <cstdint>
@@ -69,7 +70,10 @@ constexpr int kWStage = kBN * kKC / 2;   // packed bytes per (tile, chunk): 8192
 constexpr int kMaxExperts = 64;
 constexpr int kMaxGroupMsd = 512;        // expand_kernel: at most 16 values per lane
 
-enum Variant { kMsd = 0, kDeq = 1 };
+// kDeqBf16: the dequant variant with bf16 x, scale and y (the INT4 + BF16
+// pairing of the Humming article, aihirek.info).  Its buffers travel in the
+// same __half-typed fields as bit patterns; the kernels read them as bf16.
+enum Variant { kMsd = 0, kDeq = 1, kDeqBf16 = 2 };
 
 // Combine weights of equation 10 (denominators read as 7.49, 7.49*14.98,
 // 7.49*14.98^2: the page prints them with the multiplication sign lost).
@@ -126,6 +130,7 @@ struct GemmParams {
 template <int VAR, int TT, int ST, int WST, int NCONV, int NEPI, int NISS, bool SEPI>
 struct GemmCfg {
     static constexpr bool kIsMsd = VAR == kMsd;
+    static constexpr bool kBf16 = VAR == kDeqBf16;
     static constexpr bool kGroupAcc = kIsMsd || SEPI;      // per-group accumulators + per-group epilogue
     static constexpr int kVals = kIsMsd ? 3 : 1;           // accumulators per token (Y1..Y3 or y)
     static constexpr int kMmaN = kVals * TT;
@@ -174,6 +179,9 @@ struct GemmCfg {
                   "stages must split evenly over the groups");
     static_assert(NISS == 1 || NISS == 2 || NISS == 4, "1, 2 or 4 MMA issuers");
     static_assert(!SEPI || !kIsMsd, "SEPI is a DEQUANT option");
+    // bf16 keeps 8 significant bits: a product scale * w does not fit, so the
+    // weights stay exact and the scale is applied to the fp32 group sums
+    static_assert(!kBf16 || SEPI, "the bf16 variant applies the scale in the epilogue");
     static_assert(!kEpiRR || (kGroupAcc && kNBuf % NEPI == 0), "round-robin epilogue needs per-group buffers");
 };
 
@@ -220,6 +228,40 @@ __device__ __forceinline__ void int4_to_half2x4_scaled(uint32_t q, __half2 s2, u
         const __half2 v = __hmul2(*reinterpret_cast<__half2*>(&out4[i]), s2);
         out4[i] = pack_half2_bits(v);
     }
+}
+
+// Eight int4 weights of one packed word -> four bf16 pairs (w exactly), the
+// same K offsets as int4_to_half2x4.  bfloat16 is the upper half of a
+// binary32 (8 exponent bits, 7 fraction bits), so 0x4300 | u is 128 + u
+// (the fraction's unit at 128 is 1) and (128 + u) - 136 = w is exact.  A
+// nibble above bit 3 of a half would reach the exponent, so each pair is
+// shifted down first.  11 instructions.
+__device__ __forceinline__ void int4_to_bf162x4(uint32_t q, uint32_t* out4)
+{
+    const __nv_bfloat162 k136 = __halves2bfloat162(__ushort_as_bfloat16(0x4308), __ushort_as_bfloat16(0x4308));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t h = ((q >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
+        const __nv_bfloat162 w = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&h), k136);
+        out4[i] = *reinterpret_cast<const uint32_t*>(&w);
+    }
+}
+
+// One scale element of a call: fp16, or (BF) the bf16 bit pattern kept in
+// the same 16 bits.
+template <bool BF>
+__device__ __forceinline__ float load_elem(const __half* p)
+{
+    if constexpr (BF) return __uint_as_float(static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(p)) << 16);
+    else return __half2float(*p);
+}
+
+// One y element, rounded to nearest even: fp16, or (BF) bf16.
+template <bool BF>
+__device__ __forceinline__ void store_elem(__half* p, float v)
+{
+    if constexpr (BF) *reinterpret_cast<__nv_bfloat16*>(p) = __float2bfloat16_rn(v);
+    else *p = __float2half_rn(v);
 }
 
 // Eight int4 weights of one packed word -> two words of four signed int8 in
@@ -556,7 +598,8 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
         // that reconverges after every MMA roughly doubles the issue cost of
         // each one.
         if (q < issuers && lane == 0) {
-            constexpr uint32_t idesc = C::kIsMsd ? idesc_s8_s32(C::kMmaN) : idesc_f16_f32(C::kMmaN);
+            constexpr uint32_t idesc = C::kIsMsd ? idesc_s8_s32(C::kMmaN)
+                                                 : (C::kBf16 ? idesc_bf16_f32(C::kMmaN) : idesc_f16_f32(C::kMmaN));
             constexpr int kSteps = C::kIsMsd ? 4 : 8;         // MMA K steps per 128-deep chunk
             constexpr int kStepK = kKC / kSteps;
             // group bookkeeping without divisions in the step loop: K steps
@@ -697,10 +740,17 @@ W4A16_ROLE_UNROLL
 W4A16_ROLE_UNROLL
                 for (int p = 0; p < 4; ++p) {
                     uint32_t o[16];
-                    int4_to_half2x4(q[p].x, o + 0);
-                    int4_to_half2x4(q[p].y, o + 4);
-                    int4_to_half2x4(q[p].z, o + 8);
-                    int4_to_half2x4(q[p].w, o + 12);
+                    if constexpr (C::kBf16) {
+                        int4_to_bf162x4(q[p].x, o + 0);
+                        int4_to_bf162x4(q[p].y, o + 4);
+                        int4_to_bf162x4(q[p].z, o + 8);
+                        int4_to_bf162x4(q[p].w, o + 12);
+                    } else {
+                        int4_to_half2x4(q[p].x, o + 0);
+                        int4_to_half2x4(q[p].y, o + 4);
+                        int4_to_half2x4(q[p].z, o + 8);
+                        int4_to_half2x4(q[p].w, o + 12);
+                    }
                     tmem_st16(a_addr + 16 * p, o);
                 }
             } else {
@@ -760,7 +810,7 @@ W4A16_ROLE_UNROLL
                 am_next[v] = (C::kIsMsd && j0 < ngroups && tok < nt)
                                  ? __ldg(P.amax + static_cast<size_t>(grp0 + j0) * P.M + tc.t0 + tok) : 0.f;
             }
-            if (j0 < ngroups && n_ok && sc_e) sc_next = __half2float(sc_e[static_cast<size_t>(grp0 + j0) * P.N + n]);
+            if (j0 < ngroups && n_ok && sc_e) sc_next = load_elem<C::kBf16>(sc_e + static_cast<size_t>(grp0 + j0) * P.N + n);
             float* am_ring = amax_sm + (warp - C::kEpiWarp0) * 2 * TT;
             for (int j = j0, jj = 0; j < ngroups; j += jstep, ++jj) {
                 const int grp = grp0 + j;
@@ -782,7 +832,7 @@ W4A16_ROLE_UNROLL
                                 tok < nt ? __ldg(P.amax + static_cast<size_t>(grp + jstep) * P.M + tc.t0 + tok) : 0.f;
                         }
                     }
-                    if (n_ok && sc_e) sc_next = __half2float(sc_e[static_cast<size_t>(grp + jstep) * P.N + n]);
+                    if (n_ok && sc_e) sc_next = load_elem<C::kBf16>(sc_e + static_cast<size_t>(grp + jstep) * P.N + n);
                 }
                 if (C::kIsMsd) __syncwarp();
                 if (ok && !mbar_wait(smem_addr(&accfull_bar[ab]), abph, tmo, P.status, abort_flag)) ok = false;
@@ -860,7 +910,7 @@ W4A16_ROLE_UNROLL
             if (ok && P.splits == 1 && P.write_y && n_ok && (!C::kEpiRR || eg == 0)) {
 #pragma unroll
                 for (int t = 0; t < TE; ++t)
-                    if (tb + t < nt) P.y[static_cast<size_t>(tc.t0 + tb + t) * P.N + n] = __float2half_rn(acc[t]);
+                    if (tb + t < nt) store_elem<C::kBf16>(P.y + static_cast<size_t>(tc.t0 + tb + t) * P.N + n, acc[t]);
             }
         } else {
             // one accumulator over all of K per issuer (scales applied by the
@@ -894,7 +944,7 @@ W4A16_ROLE_UNROLL
 #pragma unroll
                         for (int k = 0; k < 16; ++k)
                             if (tb + 16 * c + k < nt)
-                                P.y[static_cast<size_t>(tc.t0 + tb + 16 * c + k) * P.N + n] = __float2half_rn(v[k]);
+                                store_elem<C::kBf16>(P.y + static_cast<size_t>(tc.t0 + tb + 16 * c + k) * P.N + n, v[k]);
                     }
                 }
                 tc_fence_before();
@@ -942,7 +992,7 @@ W4A16_ROLE_UNROLL
                 if (t >= nt || nn >= P.N) continue;
                 float sum = 0.f;
                 for (int sp = 0; sp < S; ++sp) sum += red[sp * per + el];
-                P.y[static_cast<size_t>(tc.t0 + t) * P.N + nn] = __float2half_rn(sum);
+                store_elem<C::kBf16>(P.y + static_cast<size_t>(tc.t0 + t) * P.N + nn, sum);
             }
         }
         if (warp == C::kEpiWarp0 && lane == 0) W4A16_TRACE_AT(55);

@@ -20,9 +20,10 @@
 //    loads, four in flight per lane); rows without an entry are zero.
 //  * moe_combine_kernel: y[t] = sum_j w[t][j] * y_sorted[row of (t, j)], fp32
 //    sums in increasing j, fp16 out (a warp per token, four 16-byte loads in
-//    flight per lane).
+//    flight per lane); the bf16 instance reads and writes bf16.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include <cstdint>
@@ -140,7 +141,8 @@ __global__ void __launch_bounds__(256) moe_gather_kernel(const uint4* __restrict
 // y[t][c .. c+7] = sum_j w[t][j] * y_sorted[inv_pos[t*topk+j]][c .. c+7],
 // fp32 sums in increasing j (entries without a row skipped), a warp per
 // token; each lane keeps four 16-byte loads in flight (columns c, c + 256,
-// c + 512, c + 768).
+// c + 512, c + 768).  BF: y_sorted and y hold bf16 bit patterns.
+template <bool BF>
 __global__ void __launch_bounds__(256) moe_combine_kernel(const __half* __restrict__ y_sorted,
                                                           const int32_t* __restrict__ inv_pos,
                                                           const float* __restrict__ weights, int T, int topk, int N,
@@ -167,10 +169,11 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(const __half* __restri
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 if (c0 + 256 * u >= N) break;
-                const __half2* h = reinterpret_cast<const __half2*>(&v[u]);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const float2 f = __half22float2(h[q]);
+                    float2 f;
+                    if constexpr (BF) f = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(&v[u])[q]);
+                    else f = __half22float2(reinterpret_cast<const __half2*>(&v[u])[q]);
                     acc[u][2 * q] = fmaf(wj, f.x, acc[u][2 * q]);
                     acc[u][2 * q + 1] = fmaf(wj, f.y, acc[u][2 * q + 1]);
                 }
@@ -180,9 +183,13 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(const __half* __restri
         for (int u = 0; u < U; ++u) {
             if (c0 + 256 * u >= N) break;
             uint4 out;
-            __half2* o = reinterpret_cast<__half2*>(&out);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) o[q] = __floats2half2_rn(acc[u][2 * q], acc[u][2 * q + 1]);
+            for (int q = 0; q < 4; ++q) {
+                if constexpr (BF)
+                    reinterpret_cast<__nv_bfloat162*>(&out)[q] = __floats2bfloat162_rn(acc[u][2 * q], acc[u][2 * q + 1]);
+                else
+                    reinterpret_cast<__half2*>(&out)[q] = __floats2half2_rn(acc[u][2 * q], acc[u][2 * q + 1]);
+            }
             *reinterpret_cast<uint4*>(y + static_cast<size_t>(t) * N + c0 + 256 * u) = out;
         }
     }
