@@ -45,6 +45,10 @@ def _load():
         lib.oracle_msd_combine.argtypes = [P, P, P, I, I, I, I, P]
         lib.oracle_msd.argtypes = [P, P, P, I, I, I, I, I, P]
         lib.oracle_msd_at.argtypes = [P, P, P, I, I, I, I, I, P, P, I, P]
+        lib.oracle_msd_expand_steps.argtypes = [P, I, I, I, I, I, P, P]
+        lib.oracle_msd_yint_planes.argtypes = [P, I, P, I, I, I, I, P]
+        lib.oracle_msd_steps.argtypes = [P, P, P, I, I, I, I, I, I, P]
+        lib.oracle_msd_at_steps.argtypes = [P, P, P, I, I, I, I, I, I, P, P, I, P]
         lib.oracle_dequant.argtypes = [P, P, P, I, I, I, I, P]
         lib.oracle_dequant_at.argtypes = [P, P, P, I, I, I, I, P, P, I, P]
         lib.oracle_bf16_to_double.restype = ctypes.c_double
@@ -149,6 +153,58 @@ def msd(x: np.ndarray, wp: np.ndarray, scale: np.ndarray, g: int,
     _check(_load().oracle_msd(_ptr(x), _ptr(wp), _ptr(scale), M, K, N, g, mode, _ptr(y)),
            "msd")
     return y
+
+
+def msd_expand_steps(x: np.ndarray, g: int, steps: int, mode: int = MODE_FP32):
+    """Equations 1-8 with `steps` digits (reading R16 of the C file): returns
+    (amax [M, K/g] float64, a_int [steps, M, K] int8)."""
+    x = _c(x, np.float16)
+    M, K = x.shape
+    amax = np.empty((M, K // g), np.float64)
+    a = np.empty((steps, M, K), np.int8)
+    _check(_load().oracle_msd_expand_steps(_ptr(x), M, K, g, mode, steps, _ptr(amax), _ptr(a)),
+           "msd_expand_steps")
+    return amax, a
+
+
+def msd_yint_planes(a: np.ndarray, wp: np.ndarray, N: int, g: int) -> np.ndarray:
+    """Equation 9 per group for any number of digit planes: a [S, M, K] ->
+    Y_int [S, M, K/g, N] int64."""
+    a = _c(a, np.int8)
+    wp = _c(wp, np.uint8)
+    S, M, K = a.shape
+    y = np.empty((S, M, K // g, N), np.int64)
+    _check(_load().oracle_msd_yint_planes(_ptr(a), S, _ptr(wp), M, K, N, g, _ptr(y)), "msd_yint_planes")
+    return y
+
+
+def msd_steps(x, wp, scale, g, steps: int, mode: int = MODE_FP32) -> np.ndarray:
+    """MSD with `steps` unfold steps (R16): y [M, N] float64."""
+    x = _c(x, np.float16)
+    wp = _c(wp, np.uint8)
+    scale = _c(scale, np.float16)
+    M, K = x.shape
+    N = wp.shape[1]
+    y = np.empty((M, N), np.float64)
+    _check(_load().oracle_msd_steps(_ptr(x), _ptr(wp), _ptr(scale), M, K, N, g, mode, steps, _ptr(y)),
+           "msd_steps")
+    return y
+
+
+def msd_at_steps(x, wp, scale, g, steps: int, rows, cols, mode: int = MODE_FP32) -> np.ndarray:
+    """MSD with `steps` unfold steps at y[rows[i], cols[i]] only (float64)."""
+    x = _c(x, np.float16)
+    wp = _c(wp, np.uint8)
+    scale = _c(scale, np.float16)
+    M, K = x.shape
+    N = wp.shape[1]
+    order, r, c = _sorted_pairs(rows, cols)
+    out = np.empty(r.size, np.float64)
+    _check(_load().oracle_msd_at_steps(_ptr(x), _ptr(wp), _ptr(scale), M, K, N, g, mode, steps,
+                                       _ptr(r), _ptr(c), r.size, _ptr(out)), "msd_at_steps")
+    res = np.empty_like(out)
+    res[order] = out
+    return res
 
 
 def _sorted_pairs(rows, cols):

@@ -35,6 +35,7 @@
  *       and y is rounded to binary16 (round-to-nearest-even) once at the end.
  *   R13, R14  the routing prep of the grouped form (see oracle_moe_align).
  *   R15  bf16 activations for the dequant form (see oracle_dequant_bf16).
+ *   R16  MSD with S = 2..4 unfold steps (see expand_row_steps).
  *
  * Build: gcc -O2 -fopenmp -ffp-contract=off -fno-fast-math -fPIC -shared
  * (binary32 arithmetic must stay IEEE single with no FMA contraction).
@@ -312,6 +313,180 @@ int oracle_msd_at(const uint16_t* x, const uint8_t* wp, const uint16_t* scale,
                 acc = merge_y(y1, y2, y3, amax[gi], s) + acc;
             }
             y[i] = acc;
+        }
+        free(amax);
+        free(a);
+    }
+    return bad ? -3 : 0;
+}
+
+/* ---------------------------------------------------------------------- */
+/* MSD with S unfold steps.  Section 7 of the same page ("性能分析") notes    */
+/* that the gain varies with the number of MSD unfold steps; section 4.1    */
+/* gives three.  Reading R16: an S-step expansion runs the same residual     */
+/* recursion (eq. 2-7) for S digits, tmp_{i+1} = (tmp_i - A_i) * 14.98 and   */
+/* A_{i+1} = round(tmp_{i+1}), so its digits are the first S digits of any   */
+/* longer expansion; eq. 10 gets one term per digit, Y_i divided by          */
+/* 7.49 * 14.98^(i-1) (extending R1).  A_max, R2-R7 are unchanged.  These    */
+/* functions stand beside the three-step ones above and do not replace them. */
+/* ---------------------------------------------------------------------- */
+
+#define ORACLE_MAX_STEPS 8
+
+/* eq. 1-7 with S digits for one row (mode 0 binary32, 1 binary64).
+ * a: digit i of element k at a[i * plane + k]. */
+static void expand_row_steps(const uint16_t* xrow, int K, int g, int mode, int S,
+                             double* amax_row, int8_t* a, size_t plane)
+{
+    int G = K / g;
+    for (int gi = 0; gi < G; ++gi) {
+        const uint16_t* xg = xrow + (size_t)gi * g;
+        double am = 0.0;                                   /* eq. 1, R2 */
+        for (int j = 0; j < g; ++j) {
+            double v = fabs(oracle_half_to_double(xg[j]));
+            if (v > am) am = v;
+        }
+        amax_row[gi] = am;
+        for (int j = 0; j < g; ++j) {
+            int k = gi * g + j;
+            if (am == 0.0) {                               /* R5 */
+                for (int i = 0; i < S; ++i) a[(size_t)i * plane + k] = 0;
+                continue;
+            }
+            if (mode == 0) {
+                float xf = (float)oracle_half_to_double(xg[j]);
+                float amf = (float)am;
+                float t = (7.49f * xf) / amf;              /* eq. 2 */
+                for (int i = 0; i < S; ++i) {
+                    float A = rintf(t);                    /* eq. 3, 5, 7, ... */
+                    a[(size_t)i * plane + k] = (int8_t)A;
+                    t = (t - A) * 14.98f;                  /* eq. 4, 6, ... */
+                }
+            } else {
+                double t = (7.49 * oracle_half_to_double(xg[j])) / am;
+                for (int i = 0; i < S; ++i) {
+                    double A = rint(t);
+                    a[(size_t)i * plane + k] = (int8_t)A;
+                    t = (t - A) * 14.98;
+                }
+            }
+        }
+    }
+}
+
+/* a: [S][M][K]; amax: [M][G]. */
+int oracle_msd_expand_steps(const uint16_t* x, int M, int K, int g, int mode, int S,
+                            double* amax, int8_t* a)
+{
+    if (g <= 0 || K % g || S < 1 || S > ORACLE_MAX_STEPS) return -1;
+    int G = K / g;
+    for (int m = 0; m < M; ++m)
+        expand_row_steps(x + (size_t)m * K, K, g, mode, S, amax + (size_t)m * G,
+                         a + (size_t)m * K, (size_t)M * K);
+    return 0;
+}
+
+/* eq. 9 for S planes: a [S][M][K] -> yint [S][M][G][N], exact in int64. */
+int oracle_msd_yint_planes(const int8_t* a, int S, const uint8_t* wp, int M, int K, int N,
+                           int g, int64_t* yint)
+{
+    if (g <= 0 || K % g || S < 1) return -1;
+    int G = K / g;
+    for (int r = 0; r < S; ++r)
+        for (int m = 0; m < M; ++m) {
+            const int8_t* ar = a + ((size_t)r * M + m) * K;
+            for (int gi = 0; gi < G; ++gi) {
+                int64_t* out = yint + (((size_t)r * M + m) * G + gi) * N;
+#pragma omp parallel for schedule(static)
+                for (int n = 0; n < N; ++n) {
+                    int64_t s = 0;
+                    for (int k = gi * g; k < (gi + 1) * g; ++k)
+                        s += (int64_t)ar[k] * weight_at(wp, N, k, n);
+                    out[n] = s;
+                }
+            }
+        }
+    return 0;
+}
+
+/* eq. 10 with S terms (R16): (sum_i Y_i / (7.49 * 14.98^(i-1))) * A_max *
+ * scale, the terms added in increasing i. */
+static double merge_y_steps(const int64_t* yi, int S, double amax, double scale)
+{
+    double den = 7.49, sum = 0.0;
+    for (int i = 0; i < S; ++i) {
+        sum = sum + (double)yi[i] / den;
+        den = den * 14.98;
+    }
+    return sum * amax * scale;
+}
+
+/* One output (m, n) from a row's digits a [S][K] (plane stride K). */
+static double msd_out_steps(const int8_t* a, int S, const double* amax, const uint8_t* wp,
+                            const uint16_t* scale, int K, int N, int g, int n)
+{
+    int G = K / g;
+    double acc = 0.0;
+    for (int gi = 0; gi < G; ++gi) {
+        int64_t yi[ORACLE_MAX_STEPS];
+        for (int i = 0; i < S; ++i) yi[i] = 0;
+        for (int k = gi * g; k < (gi + 1) * g; ++k) {
+            int w = weight_at(wp, N, k, n);
+            for (int i = 0; i < S; ++i) yi[i] += (int64_t)a[(size_t)i * K + k] * w;
+        }
+        double s = oracle_half_to_double(scale[(size_t)gi * N + n]);
+        acc = merge_y_steps(yi, S, amax[gi], s) + acc;     /* eq. 11 */
+    }
+    return acc;
+}
+
+/* All steps with S digits: y [M][N] binary64. */
+int oracle_msd_steps(const uint16_t* x, const uint8_t* wp, const uint16_t* scale,
+                     int M, int K, int N, int g, int mode, int S, double* y)
+{
+    if (g <= 0 || K % g || S < 1 || S > ORACLE_MAX_STEPS) return -1;
+    int G = K / g;
+    double* amax = (double*)malloc(sizeof(double) * (size_t)G);
+    int8_t* a = (int8_t*)malloc((size_t)S * K);
+    if (!amax || !a) { free(amax); free(a); return -2; }
+    for (int m = 0; m < M; ++m) {
+        expand_row_steps(x + (size_t)m * K, K, g, mode, S, amax, a, (size_t)K);
+#pragma omp parallel for schedule(static)
+        for (int n = 0; n < N; ++n)
+            y[(size_t)m * N + n] = msd_out_steps(a, S, amax, wp, scale, K, N, g, n);
+    }
+    free(amax);
+    free(a);
+    return 0;
+}
+
+/* The same, only at the listed (row, column) pairs. */
+int oracle_msd_at_steps(const uint16_t* x, const uint8_t* wp, const uint16_t* scale,
+                        int M, int K, int N, int g, int mode, int S,
+                        const int32_t* rows, const int32_t* cols, int count, double* y)
+{
+    if (g <= 0 || K % g || S < 1 || S > ORACLE_MAX_STEPS) return -1;
+    int G = K / g;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double* amax = (double*)malloc(sizeof(double) * (size_t)G);
+        int8_t* a = (int8_t*)malloc((size_t)S * K);
+        int last_row = -1;
+#pragma omp for schedule(static)
+        for (int i = 0; i < count; ++i) {
+            int m = rows[i], n = cols[i];
+            if (!amax || !a || m < 0 || m >= M || n < 0 || n >= N) {
+                y[i] = NAN;
+#pragma omp atomic write
+                bad = 1;
+                continue;
+            }
+            if (m != last_row) {
+                expand_row_steps(x + (size_t)m * K, K, g, mode, S, amax, a, (size_t)K);
+                last_row = m;
+            }
+            y[i] = msd_out_steps(a, S, amax, wp, scale, K, N, g, n);
         }
         free(amax);
         free(a);

@@ -423,3 +423,110 @@ def test_dequant_bf16_equals_fp16_oracle_on_shared_values():
     y16 = oracle.dequant(xi.astype(np.float16), c.wp[0], si.astype(np.float16), g)
     yb = oracle.dequant_bf16(_to_bf16_bits(xi), c.wp[0], _to_bf16_bits(si), g)
     np.testing.assert_array_equal(y16, yb)
+
+
+# ---------------------------------------------------------------- MSD with S unfold steps (reading R16)
+
+def _golden_steps():
+    with open(os.path.join(GOLDEN, "msd_worked_example_steps.json")) as f:
+        return json.load(f)
+
+
+@pytest.mark.parametrize("mode", [oracle.MODE_FP32, oracle.MODE_FP64])
+def test_worked_example_four_digits(mode):
+    """The hand-worked example carried one residual step further: the fourth
+    digit, its Y, and the 2- and 4-step outputs against their bounds."""
+    ex, base = _golden_steps(), _golden()
+    g = ex["g"]
+    x = np.array([ex["x"]], dtype=np.float16)
+    w = np.array(ex["w"], dtype=np.int8)
+    scale = np.array([ex["scale"]], dtype=np.float16)
+    amax, a = oracle.msd_expand_steps(x, g, 4, mode)
+    assert amax[0, 0] == base["amax"]
+    assert [a[i, 0].tolist() for i in range(4)] == [base["A1"], base["A2"], base["A3"], ex["A4"]]
+    yint = oracle.msd_yint_planes(a, pack_int4(w), w.shape[1], g)
+    assert [yint[i, 0, 0].tolist() for i in range(4)] == [base["Y1"], base["Y2"], base["Y3"], ex["Y4"]]
+    for S, key in ((2, "2step"), (4, "4step")):
+        y = oracle.msd_steps(x, pack_int4(w), scale, g, S, mode)
+        np.testing.assert_allclose(y[0], ex["y_msd_" + key], rtol=1e-12, atol=0)
+        assert np.all(np.abs(y[0] - np.array(base["y_exact"])) <= np.array(ex["truncation_bound_" + key]))
+
+
+@pytest.mark.parametrize("mode", [oracle.MODE_FP32, oracle.MODE_FP64])
+def test_steps_are_prefixes_and_match_the_three_step_oracle(mode):
+    """An S-step expansion's digits are the first S digits of a longer one
+    (the recursion does not look ahead), and S = 3 equals the separately
+    written three-step functions bit for bit (digits, A_max and y)."""
+    rng = np.random.default_rng(21)
+    for g in (32, 128):
+        x = _adversarial_x(rng, 8, 512, g)
+        amax4, a4 = oracle.msd_expand_steps(x, g, 4, mode)
+        for S in (1, 2, 3):
+            amax, a = oracle.msd_expand_steps(x, g, S, mode)
+            assert np.array_equal(amax, amax4)
+            assert np.array_equal(a, a4[:S])
+        amax3, a3 = oracle.msd_expand(x, g, mode)
+        assert np.array_equal(amax3, amax4) and np.array_equal(a3, a4[:3])
+    c = make_case(5, 256, 40, 64, seed=5)
+    assert np.array_equal(oracle.msd_steps(c.x, c.wp[0], c.scale[0], 64, 3, mode),
+                          oracle.msd(c.x, c.wp[0], c.scale[0], 64, mode))
+
+
+@pytest.mark.parametrize("mode", [oracle.MODE_FP32, oracle.MODE_FP64])
+@pytest.mark.parametrize("S", [1, 2, 3, 4])
+def test_steps_digits_and_reconstruction(mode, S):
+    """Every digit |A_i| <= 7, and 7.49*x/A_max = sum_i A_i/14.98^(i-1) +
+    r/14.98^(S-1) with |r| <= 0.5.  Binary32 adds the rounding of tmp1 (at
+    most 7.49 * 2^-23 plus the gap between 7.49f and 7.49) once."""
+    rng = np.random.default_rng(31 + S)
+    g = 64
+    x = _adversarial_x(rng, 8, 256, g)
+    amax, a = oracle.msd_expand_steps(x, g, S, mode)
+    assert np.abs(a).max() <= 7
+    xd = x.astype(np.float64)
+    am = np.repeat(amax, g, axis=1)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        t = np.where(am > 0, 7.49 * xd / am, 0.0)
+    rec = sum(a[i] / 14.98 ** i for i in range(S))
+    slack = 1e-12 if mode == oracle.MODE_FP64 else 2e-6
+    assert np.abs(t - rec).max() <= 0.5 / 14.98 ** (S - 1) + slack
+
+
+@pytest.mark.parametrize("mode", [oracle.MODE_FP32, oracle.MODE_FP64])
+def test_steps_within_their_truncation_bounds_and_shrinking(mode):
+    """y_S stays within sum_g A_max * 0.5/(7.49 * 14.98^(S-1)) * |scale| *
+    sum|W| of the exact GEMM, and more steps give a smaller error (the
+    accuracy side of the knob)."""
+    g = 64
+    c = make_case(6, 512, 80, g, seed=61, keep_w=True)
+    c.x[2, :g] = 0
+    ye = _exact_gemm(c.x, c.w[0], c.scale[0], g)
+    K, N = c.w[0].shape
+    absw = np.abs(c.w[0].astype(np.float64)).reshape(K // g, g, N).sum(axis=1)
+    mag = None
+    errs = []
+    for S in (1, 2, 3, 4):
+        amax, _ = oracle.msd_expand_steps(c.x, g, S, mode)
+        mag = amax @ (np.abs(c.scale[0].astype(np.float64)) * absw)
+        y = oracle.msd_steps(c.x, c.wp[0], c.scale[0], g, S, mode)
+        bound = mag * 0.5 / (7.49 * 14.98 ** (S - 1))
+        slack = 1e-12 if mode == oracle.MODE_FP64 else mag * 2e-6 / 7.49
+        assert np.all(np.abs(y - ye) <= bound + slack)
+        errs.append(np.abs(y - ye).max())
+    assert errs[0] > errs[1] > errs[2] > errs[3] > 0
+
+
+def test_yint_planes_match_integer_gemm_and_sampled_steps_match_full():
+    c = make_case(4, 256, 48, 64, seed=78, keep_w=True)
+    amax, a = oracle.msd_expand_steps(c.x, 64, 4)
+    yint = oracle.msd_yint_planes(a, c.wp[0], 48, 64)
+    w = c.w[0].astype(np.int64)
+    for r in range(4):
+        for gi in range(4):
+            ref = a[r].astype(np.int64)[:, gi * 64:(gi + 1) * 64] @ w[gi * 64:(gi + 1) * 64]
+            assert np.array_equal(yint[r, :, gi], ref)
+    rows = np.array([0, 3, 1, 3, 2])
+    cols = np.array([47, 0, 5, 9, 30])
+    for S in (2, 4):
+        full = oracle.msd_steps(c.x, c.wp[0], c.scale[0], 64, S)
+        assert np.array_equal(oracle.msd_at_steps(c.x, c.wp[0], c.scale[0], 64, S, rows, cols), full[rows, cols])
