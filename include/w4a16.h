@@ -68,8 +68,16 @@ typedef enum {
 
 /* Operation selector for w4a16_workspace_size, w4a16_grouped_matmul and
  * the routed (moe) entry points.  W4A16_OP_DEQUANT_BF16 is the dequant
- * variant with bf16 x, scale and y (see w4a16_dequant_matmul_bf16). */
-enum { W4A16_OP_MSD = 0, W4A16_OP_DEQUANT = 1, W4A16_OP_DEQUANT_BF16 = 2 };
+ * variant with bf16 x, scale and y (see w4a16_dequant_matmul_bf16);
+ * W4A16_OP_MSD_2STEP / _4STEP are MSD with 2 or 4 unfold steps instead of
+ * 3 (see w4a16_msd_matmul_steps). */
+enum {
+    W4A16_OP_MSD = 0,
+    W4A16_OP_DEQUANT = 1,
+    W4A16_OP_DEQUANT_BF16 = 2,
+    W4A16_OP_MSD_2STEP = 3,
+    W4A16_OP_MSD_4STEP = 4
+};
 
 /* Bits of the device status word kept at the start of every workspace. */
 enum { W4A16_DEVICE_TIMEOUT = 1u, W4A16_DEVICE_BAD_EXPERT = 2u };
@@ -124,6 +132,21 @@ w4a16_status w4a16_msd_matmul(const void* x, const void* w_packed, const void* s
                               void* workspace, size_t workspace_bytes,
                               w4a16_stream_t stream);
 
+/* MSD with a chosen number of unfold steps S (2, 3 or 4): the residual
+ * recursion of section 4.1 (tmp_{i+1} = (tmp_i - A_i) * 14.98f, A_{i+1} =
+ * round(tmp_{i+1}), binary32) runs for S digits, and equation 10 gets one
+ * term per digit, Y_i / (7.49 * 14.98^(i-1)).  Section 7 of the same page
+ * notes that the speed-up varies with the number of unfold steps: fewer
+ * steps do less integer work and truncate at 0.5 / (7.49 * 14.98^(S-1)) of
+ * A_max * |scale| * sum|W| per group instead of 0.5 / (7.49 * 14.98^2).
+ * S = 3 is w4a16_msd_matmul.  Arguments as w4a16_msd_matmul, the workspace
+ * sized for W4A16_OP_MSD_2STEP / W4A16_OP_MSD / W4A16_OP_MSD_4STEP.  Any
+ * other S returns W4A16_ERR_INVALID_ARG. */
+w4a16_status w4a16_msd_matmul_steps(int steps, const void* x, const void* w_packed,
+                                    const void* scale, int M, int K, int N, int group_size,
+                                    void* y, void* workspace, size_t workspace_bytes,
+                                    w4a16_stream_t stream);
+
 /* Direct dequant variant: W' = fp16(scale * W) in registers, y = x . W' on
  * the fp16 tensor cores with fp32 accumulation, y rounded to fp16 once.
  * Arguments as w4a16_msd_matmul (workspace sized for W4A16_OP_DEQUANT). */
@@ -154,7 +177,7 @@ w4a16_status w4a16_dequant_matmul_bf16(const void* x, const void* w_packed, cons
 /* Grouped-expert (MoE) form: expert e multiplies the contiguous token rows
  * offsets[e] .. offsets[e+1]-1 of x by its own weights (the dense and MoE
  * scheduling Humming describes, aihirek.info "Humming ..." article).
- *   op         W4A16_OP_MSD, W4A16_OP_DEQUANT or W4A16_OP_DEQUANT_BF16
+ *   op         any W4A16_OP_* code
  *   x          device fp16 [T][K] (bf16 for W4A16_OP_DEQUANT_BF16), tokens
  *              sorted by expert
  *   w_packed   host array of E device pointers (each from w4a16_repack)
@@ -243,6 +266,14 @@ w4a16_status w4a16_msd_debug_yint(const void* x, const void* w_packed, int M, in
                                   int N, int group_size, int m0, int m1, int n0, int n1,
                                   int32_t* yint, float* amax, void* workspace,
                                   size_t workspace_bytes, w4a16_stream_t stream);
+
+/* The same window for S = 2, 3 or 4 unfold steps (w4a16_msd_matmul_steps):
+ * yint device int32 [S][m1-m0][K/g][n1-n0]; workspace sized for the op of S. */
+w4a16_status w4a16_msd_debug_yint_steps(int steps, const void* x, const void* w_packed,
+                                        int M, int K, int N, int group_size, int m0, int m1,
+                                        int n0, int n1, int32_t* yint, float* amax,
+                                        void* workspace, size_t workspace_bytes,
+                                        w4a16_stream_t stream);
 
 /* MSD matmul for callers that cannot allocate device memory.
  * No counterpart in the paper: this entry point exists for callers that have

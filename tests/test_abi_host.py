@@ -55,6 +55,10 @@ def test_workspace_sizes(lib):
     assert msd - deq >= 3 * 16 * 4096 + 32 * 16 * 4
     assert lib.w4a16_workspace_size(lib.OP_DEQUANT, 0, 256, 256, 64) >= 256
     assert lib.w4a16_workspace_size(lib.OP_MSD, 4096, 4096, 14336, 128, E=8) >= 3 * 4096 * 4096
+    # MSD with S unfold steps holds S digit planes (S * M * K bytes)
+    m2, m3, m4 = (lib.w4a16_workspace_size(op, 4096, 4096, 4096, 128)
+                  for op in (lib.OP_MSD_2STEP, lib.OP_MSD, lib.OP_MSD_4STEP))
+    assert m3 - m2 == 4096 * 4096 and m4 - m3 == 4096 * 4096
     # the bf16 dequant variant needs what the fp16 one needs
     for M in (1, 8, 16, 4096):
         assert lib.w4a16_workspace_size(lib.OP_DEQUANT_BF16, M, 4096, 14336, 128) == \
@@ -68,7 +72,8 @@ def test_workspace_sizes(lib):
     ((0, -1, 4096, 4096, 128), 1),      # negative M
     ((0, 16, 4096, 4096, 1024), 2),     # MSD group larger than 512
     ((7, 16, 4096, 4096, 128), 1),      # bad op
-    ((3, 16, 4096, 4096, 128), 1),      # first code past the bf16 dequant op
+    ((5, 16, 4096, 4096, 128), 1),      # first code past the MSD step variants
+    ((4, 16, 4096, 4096, 1024), 2),     # four-step MSD, group larger than 512
 ])
 def test_workspace_size_rejects(lib, args, code):
     with pytest.raises(lib.W4A16Error) as e:
@@ -93,6 +98,15 @@ def test_matmul_rejects_before_launch(lib):
         assert e.value.code == 2
     # M == 0 is a no-op that touches nothing
     lib.w4a16_dequant_matmul(None, None, None, 0, 256, 256, 64, None, None, 0, stream=0)
+    # MSD unfold steps other than 2, 3, 4 are rejected
+    for steps in (0, 1, 5):
+        with pytest.raises(lib.W4A16Error) as e:
+            lib.w4a16_msd_matmul_steps(steps, fake, fake, fake, 16, 256, 256, 64, fake, fake, 1 << 20, stream=0)
+        assert e.value.code == 1
+    with pytest.raises(lib.W4A16Error) as e:     # workspace sized for 3 steps is too small for 4
+        need = lib.w4a16_workspace_size(lib.OP_MSD, 64, 256, 256, 64)
+        lib.w4a16_msd_matmul_steps(4, fake, fake, fake, 64, 256, 256, 64, fake, fake, need, stream=0)
+    assert e.value.code == 3
 
 
 def test_grouped_and_debug_reject(lib):

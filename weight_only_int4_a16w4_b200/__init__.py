@@ -25,6 +25,8 @@ _lib = ctypes.CDLL(LIB_PATH)
 OP_MSD = 0
 OP_DEQUANT = 1
 OP_DEQUANT_BF16 = 2
+OP_MSD_2STEP = 3
+OP_MSD_4STEP = 4
 DEVICE_TIMEOUT = 1
 DEVICE_BAD_EXPERT = 2
 
@@ -56,6 +58,10 @@ for _name in ("w4a16_msd_matmul", "w4a16_dequant_matmul", "w4a16_dequant_matmul_
     getattr(_lib, _name).argtypes = [_P, _P, _P, _I, _I, _I, _I, _P, _P, _SZ, _P]
 _lib.w4a16_grouped_matmul.restype = _I
 _lib.w4a16_grouped_matmul.argtypes = [_I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]
+_lib.w4a16_msd_matmul_steps.restype = _I
+_lib.w4a16_msd_matmul_steps.argtypes = [_I, _P, _P, _P, _I, _I, _I, _I, _P, _P, _SZ, _P]
+_lib.w4a16_msd_debug_yint_steps.restype = _I
+_lib.w4a16_msd_debug_yint_steps.argtypes = [_I, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]
 _lib.w4a16_msd_debug_yint.restype = _I
 _lib.w4a16_msd_debug_yint.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]
 _lib.w4a16_msd_matmul_noalloc.restype = _I
@@ -159,6 +165,21 @@ def w4a16_msd_debug_yint(x, w_packed, M, K, N, group_size, m0, m1, n0, n1, yint,
     _check(_lib.w4a16_msd_debug_yint(_ptr(x), _ptr(w_packed), M, K, N, group_size, m0, m1, n0, n1, _ptr(yint),
                                      _ptr(amax), _ptr(workspace), wb, _stream(stream)),
            "w4a16_msd_debug_yint")
+
+
+def w4a16_msd_matmul_steps(steps, x, w_packed, scale, M, K, N, group_size, y, workspace, workspace_bytes=None,
+                           stream=None):
+    wb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check(_lib.w4a16_msd_matmul_steps(steps, _ptr(x), _ptr(w_packed), _ptr(scale), M, K, N, group_size, _ptr(y),
+                                       _ptr(workspace), wb, _stream(stream)), "w4a16_msd_matmul_steps")
+
+
+def w4a16_msd_debug_yint_steps(steps, x, w_packed, M, K, N, group_size, m0, m1, n0, n1, yint, amax, workspace,
+                               workspace_bytes=None, stream=None):
+    wb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check(_lib.w4a16_msd_debug_yint_steps(steps, _ptr(x), _ptr(w_packed), M, K, N, group_size, m0, m1, n0, n1,
+                                           _ptr(yint), _ptr(amax), _ptr(workspace), wb, _stream(stream)),
+           "w4a16_msd_debug_yint_steps")
 
 
 def w4a16_moe_align(topk_ids, T, topk, E, offsets, sorted_token, inv_pos, workspace, workspace_bytes=None,

@@ -43,7 +43,10 @@ constexpr int kMaxSmemOptin = 227 * 1024;   // dynamic shared memory a CTA may o
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 int cdiv(int a, int b) { return (a + b - 1) / b; }
 
-bool op_ok(int op) { return op == W4A16_OP_MSD || op == W4A16_OP_DEQUANT || op == W4A16_OP_DEQUANT_BF16; }
+bool is_msd_op(int op) { return op == W4A16_OP_MSD || op == W4A16_OP_MSD_2STEP || op == W4A16_OP_MSD_4STEP; }
+bool op_ok(int op) { return is_msd_op(op) || op == W4A16_OP_DEQUANT || op == W4A16_OP_DEQUANT_BF16; }
+// MSD digit planes of an op (the unfold steps)
+int op_steps(int op) { return op == W4A16_OP_MSD_2STEP ? 2 : (op == W4A16_OP_MSD_4STEP ? 4 : 3); }
 
 bool group_ok(int g)
 {
@@ -126,7 +129,9 @@ bool small_tile(int op, int M) { (void)op; return M <= 16; }
 int tile_tokens(int op, int M, int N)
 {
     if (small_tile(op, M)) return 16;
-    if (op == W4A16_OP_MSD) return 64;
+    // MSD: 64 tokens (2 or 3 planes), 32 with four planes (4 x 32 MMA rows
+    // keep two per-group accumulator buffers within Tensor Memory)
+    if (is_msd_op(op)) return op_steps(op) == 4 ? 32 : 64;
     if (op == W4A16_OP_DEQUANT_BF16) return 128;
     static int forced = -1;
     if (forced < 0) {
@@ -179,22 +184,38 @@ Shape grouped_shape(int op, int T, int K, int N, int g, int E)
 
 // ---------------------------------------------------------------- the CUDA-core decode GEMV
 
+// the warp-MMA GEMV's rows: S digit planes x MR tokens must fit 8 MMA rows
+int gemv_mma_max_m(int op) { return is_msd_op(op) ? 8 / op_steps(op) : 8; }
+
+// rows of the instance: 1, 2, 4 or 8 tokens, capped by the variant
 int gemv_mma_rows(int op, int M)
 {
-    if (op == W4A16_OP_MSD) return M <= 1 ? 1 : 2;
-    return M <= 1 ? 1 : (M <= 2 ? 2 : (M <= 4 ? 4 : 8));
+    const int r = M <= 1 ? 1 : (M <= 2 ? 2 : (M <= 4 ? 4 : 8));
+    const int cap = is_msd_op(op) ? (op_steps(op) == 2 ? 4 : 2) : 8;
+    return std::min(r, cap);
+}
+
+template <int VAR>
+int gemv_mma_smem_var(int MR, int M, int np, int ppg)
+{
+    // instances exist for S * MR <= 8 only
+    constexpr int S = is_msd(VAR) ? msd_steps(VAR) : 1;
+    switch (MR) {
+        case 1: return MgCfg<VAR, 1>::smem_bytes(M, np, ppg);
+        case 2: return MgCfg<VAR, 2>::smem_bytes(M, np, ppg);
+        case 4: return MgCfg<VAR, 4 * S <= 8 ? 4 : 1>::smem_bytes(M, np, ppg);
+        default: return MgCfg<VAR, 8 * S <= 8 ? 8 : 1>::smem_bytes(M, np, ppg);
+    }
 }
 
 int gemv_mma_smem(int op, int M, int K, int g)
 {
-    const int np = K / 32, ppg = g / 32;
-    if (op == W4A16_OP_MSD)
-        return gemv_mma_rows(op, M) == 1 ? MgCfg<kMsd, 1>::smem_bytes(M, np, ppg) : MgCfg<kMsd, 2>::smem_bytes(M, np, ppg);
-    switch (gemv_mma_rows(op, M)) {
-        case 1: return MgCfg<kDeq, 1>::smem_bytes(M, np, ppg);
-        case 2: return MgCfg<kDeq, 2>::smem_bytes(M, np, ppg);
-        case 4: return MgCfg<kDeq, 4>::smem_bytes(M, np, ppg);
-        default: return MgCfg<kDeq, 8>::smem_bytes(M, np, ppg);
+    const int np = K / 32, ppg = g / 32, MR = gemv_mma_rows(op, M);
+    switch (op) {
+        case W4A16_OP_MSD: return gemv_mma_smem_var<kMsd>(MR, M, np, ppg);
+        case W4A16_OP_MSD_2STEP: return gemv_mma_smem_var<kMsd2>(MR, M, np, ppg);
+        case W4A16_OP_MSD_4STEP: return gemv_mma_smem_var<kMsd4>(MR, M, np, ppg);
+        default: return gemv_mma_smem_var<kDeq>(MR, M, np, ppg);
     }
 }
 
@@ -225,10 +246,12 @@ int small_override()
 int small_kernel(int op, int M, int K, int N, int g, int E)
 {
     if (E != 1 || M < 1) return kSmallNone;
-    const bool mma_ok = g % 128 == 0 && M <= (op == W4A16_OP_MSD ? 2 : 8) &&
+    const bool mma_ok = g % 128 == 0 && M <= gemv_mma_max_m(op) &&
                         static_cast<long long>(N / 8) * sm_count() < (1ll << 31) &&
                         gemv_mma_smem(op, M, K, g) <= kMaxSmemOptin;
-    const bool cuda_ok = op != W4A16_OP_DEQUANT_BF16 && M <= 4 && static_cast<long long>(M) * K <= kGemvMaxMK;
+    // (the CUDA-core GEMV is built for fp16 dequant and three-step MSD only)
+    const bool cuda_ok = (op == W4A16_OP_DEQUANT || op == W4A16_OP_MSD) && M <= 4 &&
+                         static_cast<long long>(M) * K <= kGemvMaxMK;
     const int forced = small_override();
     if (forced == kSmallNone) return kSmallNone;
     if (forced == kSmallCuda) return cuda_ok ? kSmallCuda : kSmallNone;
@@ -252,15 +275,16 @@ WsLayout ws_layout(int op, const Shape& s, int M, int K, int N, int g, int E = 1
     (void)N;
     WsLayout L;
     size_t off = kHeaderBytes;
-    if (op == W4A16_OP_MSD) {
+    if (is_msd_op(op)) {
+        const int S = op_steps(op);
         L.xq = off;
-        off += align256(static_cast<size_t>(3) * M * K);
+        off += align256(static_cast<size_t>(S) * M * K);
         L.amax = off;
         off += align256(static_cast<size_t>(K / g) * M * 4);
         if (small_kernel(op, M, K, N, g, E) != kSmallNone) {
-            // the decode GEMV's digit records [K/32][M][28 words]
+            // the decode GEMV's digit records [K/32][M][gemv_rec_words(S)]
             L.rec = off;
-            off += align256(static_cast<size_t>(K / 32) * M * kGemvRecWords * 4);
+            off += align256(static_cast<size_t>(K / 32) * M * gemv_rec_words(S) * 4);
         }
     }
     L.total = off;
@@ -359,6 +383,23 @@ w4a16_status launch_for(int op, int TT, const CUtensorMap& map, const GemmParams
         if (TT == 16) return launch_gemm<kMsd, 16, 8, 12, 2, 2, 4, false>(map, P, grid, s);
         return launch_gemm<kMsd, 64, 4, 4, 2, 2, 1, false>(map, P, grid, s);
     }
+    if (op == W4A16_OP_MSD_2STEP) {
+        if (P.dbg_yint != nullptr) {
+            if (TT == 16) return launch_gemm<kMsd2, 16, 8, 12, 2, 1, 4, false, true>(map, P, grid, s);
+            return launch_gemm<kMsd2, 64, 4, 4, 2, 2, 1, false, true>(map, P, grid, s);
+        }
+        if (TT == 16) return launch_gemm<kMsd2, 16, 8, 12, 2, 2, 4, false>(map, P, grid, s);
+        return launch_gemm<kMsd2, 64, 4, 4, 2, 2, 1, false>(map, P, grid, s);
+    }
+    if (op == W4A16_OP_MSD_4STEP) {
+        // 4 x 16-row activation stages: 8 weight stages keep shared memory in bounds
+        if (P.dbg_yint != nullptr) {
+            if (TT == 16) return launch_gemm<kMsd4, 16, 8, 8, 2, 1, 4, false, true>(map, P, grid, s);
+            return launch_gemm<kMsd4, 32, 4, 4, 2, 2, 1, false, true>(map, P, grid, s);
+        }
+        if (TT == 16) return launch_gemm<kMsd4, 16, 8, 8, 2, 2, 4, false>(map, P, grid, s);
+        return launch_gemm<kMsd4, 32, 4, 4, 2, 2, 1, false>(map, P, grid, s);
+    }
     if (op == W4A16_OP_DEQUANT_BF16) {
         if (TT == 16) return launch_gemm<kDeqBf16, 16, 4, 12, 2, 2, 4, true>(map, P, grid, s);
         return launch_gemm<kDeqBf16, 128, 4, 4, 2, 2, 2, true>(map, P, grid, s);
@@ -368,7 +409,7 @@ w4a16_status launch_for(int op, int TT, const CUtensorMap& map, const GemmParams
     return launch_gemm<kDeq, 128, 4, 4, 2, 1, 2, false>(map, P, grid, s);
 }
 
-template <int VPL>
+template <int VPL, int S>
 cudaError_t launch_expand_vpl(int blocks, const __half* x, int M, int K, int g, int8_t* xq, float* amax,
                               cudaStream_t s)
 {
@@ -381,23 +422,36 @@ cudaError_t launch_expand_vpl(int blocks, const __half* x, int M, int K, int g, 
     attr.val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = &attr;
     cfg.numAttrs = use_pdl() ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, expand_kernel<VPL>, x, M, K, g, xq, amax);
+    return cudaLaunchKernelEx(&cfg, expand_kernel<VPL, S>, x, M, K, g, xq, amax);
 }
 
-w4a16_status launch_expand(const void* x, int M, int K, int g, int8_t* xq, float* amax, cudaStream_t s)
+template <int S>
+cudaError_t launch_expand_s(int blocks, const __half* xh, int M, int K, int g, int8_t* xq, float* amax,
+                            cudaStream_t s)
+{
+    switch (g / 32) {
+        case 1: return launch_expand_vpl<1, S>(blocks, xh, M, K, g, xq, amax, s);
+        case 2: return launch_expand_vpl<2, S>(blocks, xh, M, K, g, xq, amax, s);
+        case 4: return launch_expand_vpl<4, S>(blocks, xh, M, K, g, xq, amax, s);
+        case 8: return launch_expand_vpl<8, S>(blocks, xh, M, K, g, xq, amax, s);
+        case 12: return launch_expand_vpl<12, S>(blocks, xh, M, K, g, xq, amax, s);
+        case 16: return launch_expand_vpl<16, S>(blocks, xh, M, K, g, xq, amax, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+w4a16_status launch_expand(int op, const void* x, int M, int K, int g, int8_t* xq, float* amax, cudaStream_t s)
 {
     const long long warps = static_cast<long long>(M) * (K / g);
     const int blocks = static_cast<int>((warps + 7) / 8);
     const __half* xh = static_cast<const __half*>(x);
+    const int v = g / 32;
+    if (!(v == 1 || v == 2 || v == 4 || v == 8 || v == 12 || v == 16)) return W4A16_ERR_UNSUPPORTED;
     cudaError_t e;
-    switch (g / 32) {
-        case 1: e = launch_expand_vpl<1>(blocks, xh, M, K, g, xq, amax, s); break;
-        case 2: e = launch_expand_vpl<2>(blocks, xh, M, K, g, xq, amax, s); break;
-        case 4: e = launch_expand_vpl<4>(blocks, xh, M, K, g, xq, amax, s); break;
-        case 8: e = launch_expand_vpl<8>(blocks, xh, M, K, g, xq, amax, s); break;
-        case 12: e = launch_expand_vpl<12>(blocks, xh, M, K, g, xq, amax, s); break;
-        case 16: e = launch_expand_vpl<16>(blocks, xh, M, K, g, xq, amax, s); break;
-        default: return W4A16_ERR_UNSUPPORTED;
+    switch (op_steps(op)) {
+        case 2: e = launch_expand_s<2>(blocks, xh, M, K, g, xq, amax, s); break;
+        case 4: e = launch_expand_s<4>(blocks, xh, M, K, g, xq, amax, s); break;
+        default: e = launch_expand_s<3>(blocks, xh, M, K, g, xq, amax, s); break;
     }
     if (e != cudaSuccess) {
         (void)cudaGetLastError();
@@ -464,7 +518,9 @@ template <int VAR, int MR>
 w4a16_status launch_gemv_mma_mr(const GemvParams& P, cudaStream_t stream)
 {
     auto kern = gemv_mma_kernel<VAR, MR>;
-    const int smem = gemv_mma_smem(VAR == kMsd ? W4A16_OP_MSD : W4A16_OP_DEQUANT, P.M, P.K, P.g);
+    const int op = VAR == kMsd ? W4A16_OP_MSD : VAR == kMsd2 ? W4A16_OP_MSD_2STEP
+                 : VAR == kMsd4 ? W4A16_OP_MSD_4STEP : W4A16_OP_DEQUANT;
+    const int smem = gemv_mma_smem(op, P.M, P.K, P.g);
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
@@ -489,7 +545,7 @@ w4a16_status launch_gemv_mma_mr(const GemvParams& P, cudaStream_t stream)
     return W4A16_OK;
 }
 
-template <int NSUB>
+template <int NSUB, int S>
 cudaError_t launch_gemv_expand_n(const __half* x, int M, int K, int g, uint32_t* rec, cudaStream_t s)
 {
     const int span = NSUB * kKC;
@@ -503,7 +559,32 @@ cudaError_t launch_gemv_expand_n(const __half* x, int M, int K, int g, uint32_t*
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = use_pdl() ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, gemv_expand_kernel<NSUB>, x, M, K, g, rec);
+    return cudaLaunchKernelEx(&cfg, gemv_expand_kernel<NSUB, S>, x, M, K, g, rec);
+}
+
+template <int S>
+cudaError_t launch_gemv_expand_s(const __half* x, int M, int K, int g, uint32_t* rec, cudaStream_t s)
+{
+    switch (std::max(1, g / kKC)) {
+        case 1: return launch_gemv_expand_n<1, S>(x, M, K, g, rec, s);
+        case 2: return launch_gemv_expand_n<2, S>(x, M, K, g, rec, s);
+        case 3: return launch_gemv_expand_n<3, S>(x, M, K, g, rec, s);
+        case 4: return launch_gemv_expand_n<4, S>(x, M, K, g, rec, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+// the warp-MMA GEMV of an MSD variant, MR chosen by M
+template <int VAR>
+w4a16_status launch_gemv_mma_msd(const GemvParams& P, int op, cudaStream_t stream)
+{
+    switch (gemv_mma_rows(op, P.M)) {
+        case 1: return launch_gemv_mma_mr<VAR, 1>(P, stream);
+        case 2: return launch_gemv_mma_mr<VAR, 2>(P, stream);
+        default:
+            if constexpr (4 * msd_steps(VAR) <= 8) return launch_gemv_mma_mr<VAR, 4>(P, stream);
+            return W4A16_ERR_UNSUPPORTED;
+    }
 }
 
 w4a16_status launch_gemv(int op, bool mma, const void* x, const void* w_packed, const void* scale, int M, int K, int N,
@@ -525,24 +606,29 @@ w4a16_status launch_gemv(int op, bool mma, const void* x, const void* w_packed, 
     P.npieces = K / 32;
     P.nblk = mma ? N / 8 : cdiv(N, 32);
     P.ctas = gemv_ctas(P.nblk);
-    if (op == W4A16_OP_MSD) {
+    if (is_msd_op(op)) {
         uint32_t* rec = reinterpret_cast<uint32_t*>(wsb + L.rec);
         P.rec = rec;
         const __half* xh = static_cast<const __half*>(x);
+        if (std::max(1, g / kKC) > 4) return W4A16_ERR_UNSUPPORTED;
+        if (!mma && op != W4A16_OP_MSD) return W4A16_ERR_UNSUPPORTED;   // CUDA-core GEMV: three steps only
         cudaError_t e;
-        switch (std::max(1, g / kKC)) {
-            case 1: e = launch_gemv_expand_n<1>(xh, M, K, g, rec, stream); break;
-            case 2: e = launch_gemv_expand_n<2>(xh, M, K, g, rec, stream); break;
-            case 3: e = launch_gemv_expand_n<3>(xh, M, K, g, rec, stream); break;
-            case 4: e = launch_gemv_expand_n<4>(xh, M, K, g, rec, stream); break;
-            default: return W4A16_ERR_UNSUPPORTED;
+        switch (op_steps(op)) {
+            case 2: e = launch_gemv_expand_s<2>(xh, M, K, g, rec, stream); break;
+            case 4: e = launch_gemv_expand_s<4>(xh, M, K, g, rec, stream); break;
+            default: e = launch_gemv_expand_s<3>(xh, M, K, g, rec, stream); break;
         }
         if (e != cudaSuccess) {
             (void)cudaGetLastError();
             return W4A16_ERR_CUDA;
         }
-        if (mma) return gemv_mma_rows(op, M) == 1 ? launch_gemv_mma_mr<kMsd, 1>(P, stream)
-                                                  : launch_gemv_mma_mr<kMsd, 2>(P, stream);
+        if (mma) {
+            switch (op_steps(op)) {
+                case 2: return launch_gemv_mma_msd<kMsd2>(P, op, stream);
+                case 4: return launch_gemv_mma_msd<kMsd4>(P, op, stream);
+                default: return launch_gemv_mma_msd<kMsd>(P, op, stream);
+            }
+        }
         if (M == 1) return launch_gemv_mr<kMsd, 1>(P, stream);
         if (M == 2) return launch_gemv_mr<kMsd, 2>(P, stream);
         return launch_gemv_mr<kMsd, 4>(P, stream);
@@ -576,7 +662,7 @@ w4a16_status dense_matmul(int op, const void* x, const void* w_packed, const voi
 {
     w4a16_status st = check_shape(M, K, N, g);
     if (st != W4A16_OK) return st;
-    if (op == W4A16_OP_MSD && g > kMaxGroupMsd) return W4A16_ERR_UNSUPPORTED;
+    if (is_msd_op(op) && g > kMaxGroupMsd) return W4A16_ERR_UNSUPPORTED;
     if (M == 0) return W4A16_OK;
     const bool debug = dbg_yint != nullptr;
     if (!x || !w_packed || (!scale && !debug) || (!y && !debug) || !ws) return W4A16_ERR_INVALID_ARG;
@@ -609,13 +695,14 @@ w4a16_status dense_matmul(int op, const void* x, const void* w_packed, const voi
         if (sk != kSmallNone) return launch_gemv(op, sk == kSmallMma, x, w_packed, scale, M, K, N, g, y, ws, s, L, stream);
     }
     CUtensorMap map;
-    if (op == W4A16_OP_MSD) {
+    if (is_msd_op(op)) {
         int8_t* xq = reinterpret_cast<int8_t*>(wsb + L.xq);
         float* amax = reinterpret_cast<float*>(wsb + L.amax);
-        st = launch_expand(x, M, K, g, xq, amax, stream);
+        st = launch_expand(op, x, M, K, g, xq, amax, stream);
         if (st != W4A16_OK) return st;
         P.amax = amax;
-        if (!make_map(&map, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, 3 * M, kKC, s.TT)) return W4A16_ERR_CUDA;
+        if (!make_map(&map, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, op_steps(op) * M, kKC, s.TT))
+            return W4A16_ERR_CUDA;
     } else {
         if (!make_map(&map, x, act_dtype(op), 2, K, M, 64, s.TT)) return W4A16_ERR_CUDA;
     }
@@ -686,7 +773,7 @@ w4a16_status w4a16_workspace_size(int op, int M, int K, int N, int group_size, i
     if (E < 1 || E > kMaxExperts) return W4A16_ERR_INVALID_ARG;
     w4a16_status st = check_shape(M, K, N, group_size);
     if (st != W4A16_OK) return st;
-    if (op == W4A16_OP_MSD && group_size > kMaxGroupMsd) return W4A16_ERR_UNSUPPORTED;
+    if (is_msd_op(op) && group_size > kMaxGroupMsd) return W4A16_ERR_UNSUPPORTED;
     const Shape s = (E == 1) ? dense_shape(op, M, K, N, group_size) : grouped_shape(op, M, K, N, group_size, E);
     *bytes = ws_layout(op, s, M, K, N, group_size, E).total;
     return W4A16_OK;
@@ -728,15 +815,41 @@ w4a16_status w4a16_dequant_matmul_bf16(const void* x, const void* w_packed, cons
                         workspace_bytes, reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr, 0, 0, 0, 0);
 }
 
+namespace {
+int steps_op(int steps)
+{
+    return steps == 2 ? W4A16_OP_MSD_2STEP : steps == 3 ? W4A16_OP_MSD : steps == 4 ? W4A16_OP_MSD_4STEP : -1;
+}
+}  // namespace
+
+w4a16_status w4a16_msd_matmul_steps(int steps, const void* x, const void* w_packed, const void* scale, int M, int K,
+                                    int N, int group_size, void* y, void* workspace, size_t workspace_bytes,
+                                    w4a16_stream_t stream)
+{
+    const int op = steps_op(steps);
+    if (op < 0) return W4A16_ERR_INVALID_ARG;
+    return dense_matmul(op, x, w_packed, scale, M, K, N, group_size, y, workspace, workspace_bytes,
+                        reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr, 0, 0, 0, 0);
+}
+
+w4a16_status w4a16_msd_debug_yint_steps(int steps, const void* x, const void* w_packed, int M, int K, int N,
+                                        int group_size, int m0, int m1, int n0, int n1, int32_t* yint, float* amax,
+                                        void* workspace, size_t workspace_bytes, w4a16_stream_t stream)
+{
+    const int op = steps_op(steps);
+    if (op < 0 || !yint || !amax) return W4A16_ERR_INVALID_ARG;
+    if (m0 < 0 || m1 <= m0 || m1 > M || n0 < 0 || n1 <= n0 || n1 > N) return W4A16_ERR_INVALID_ARG;
+    // equation 9 needs no scale
+    return dense_matmul(op, x, w_packed, nullptr, M, K, N, group_size, nullptr, workspace, workspace_bytes,
+                        reinterpret_cast<cudaStream_t>(stream), yint, amax, m0, m1, n0, n1);
+}
+
 w4a16_status w4a16_msd_debug_yint(const void* x, const void* w_packed, int M, int K, int N, int group_size,
                                   int m0, int m1, int n0, int n1, int32_t* yint, float* amax, void* workspace,
                                   size_t workspace_bytes, w4a16_stream_t stream)
 {
-    if (!yint || !amax) return W4A16_ERR_INVALID_ARG;
-    if (m0 < 0 || m1 <= m0 || m1 > M || n0 < 0 || n1 <= n0 || n1 > N) return W4A16_ERR_INVALID_ARG;
-    // equation 9 needs no scale
-    return dense_matmul(W4A16_OP_MSD, x, w_packed, nullptr, M, K, N, group_size, nullptr, workspace,
-                        workspace_bytes, reinterpret_cast<cudaStream_t>(stream), yint, amax, m0, m1, n0, n1);
+    return w4a16_msd_debug_yint_steps(3, x, w_packed, M, K, N, group_size, m0, m1, n0, n1, yint, amax, workspace,
+                                      workspace_bytes, stream);
 }
 
 w4a16_status w4a16_grouped_matmul(int op, const void* x, const void* const* w_packed, const void* const* scale,
@@ -747,7 +860,7 @@ w4a16_status w4a16_grouped_matmul(int op, const void* x, const void* const* w_pa
     if (E < 1 || E > kMaxExperts) return W4A16_ERR_INVALID_ARG;
     w4a16_status st = check_shape(T, K, N, group_size);
     if (st != W4A16_OK) return st;
-    if (op == W4A16_OP_MSD && group_size > kMaxGroupMsd) return W4A16_ERR_UNSUPPORTED;
+    if (is_msd_op(op) && group_size > kMaxGroupMsd) return W4A16_ERR_UNSUPPORTED;
     if (T == 0) return W4A16_OK;
     if (!x || !w_packed || !scale || !offsets || !y || !workspace) return W4A16_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(y) || !aligned16(workspace)) return W4A16_ERR_INVALID_ARG;
@@ -770,13 +883,14 @@ w4a16_status w4a16_grouped_matmul(int op, const void* x, const void* const* w_pa
     }
     P.y = static_cast<__half*>(y);
     CUtensorMap map;
-    if (op == W4A16_OP_MSD) {
+    if (is_msd_op(op)) {
         int8_t* xq = reinterpret_cast<int8_t*>(wsb + L.xq);
         float* amax = reinterpret_cast<float*>(wsb + L.amax);
-        st = launch_expand(x, T, K, group_size, xq, amax, cs);
+        st = launch_expand(op, x, T, K, group_size, xq, amax, cs);
         if (st != W4A16_OK) return st;
         P.amax = amax;
-        if (!make_map(&map, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, 3 * T, kKC, s.TT)) return W4A16_ERR_CUDA;
+        if (!make_map(&map, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, op_steps(op) * T, kKC, s.TT))
+            return W4A16_ERR_CUDA;
     } else {
         if (!make_map(&map, x, act_dtype(op), 2, K, T, 64, s.TT)) return W4A16_ERR_CUDA;
     }

@@ -51,6 +51,9 @@ constexpr int kGemvThreads = 256;
 constexpr int kGemvWarps = kGemvThreads / 32;
 constexpr int kGemvRound = 8;                        // 16-byte loads per thread per round
 constexpr int kGemvRecWords = 28;                    // MSD record: 24 digit words, 3 sums, A_max
+// record of an MSD call with S digit planes: 8 S digit words, S sums, A_max,
+// padded to whole 16-byte vectors (S = 3: 28 words)
+__host__ __device__ constexpr int gemv_rec_words(int S) { return (9 * S + 1 + 3) / 4 * 4; }
 constexpr int kGemvMaxMK = 32768;                    // M * K bound of the shared-memory operand
 
 struct GemvParams {
@@ -129,21 +132,22 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p)
 
 // ------------------------------------------------------------------ MSD steps 1-8 for the GEMV
 
-// One warp per (row m, span of S = max(g, 128) K values); lane l holds the
-// values 4l .. 4l+3 of each 128-value sub-chunk of the span (NSUB = S / 128
-// sub-chunks).  A_max per group (g < 128: the g/4 lanes of a group reduce
-// among themselves), then the digits in IEEE binary32 with the literal
+// One warp per (row m, span of max(g, 128) K values); lane l holds the
+// values 4l .. 4l+3 of each 128-value sub-chunk of the span (NSUB = span /
+// 128 sub-chunks).  A_max per group (g < 128: the g/4 lanes of a group reduce
+// among themselves), then the S digits in IEEE binary32 with the literal
 // operation order of steps 2-7, then per 32-K piece (8 lanes) a record of
-// 28 words: word i*8 + 2j + h holds digit plane i's bytes for the piece's
-// packed word j, low (h = 0: K offsets 8j + {0, 4, 1, 5}) or high (h = 1:
-// 8j + {2, 6, 3, 7}) nibbles -- the byte order of q & 0x0F0F0F0F and
-// (q >> 4) & 0x0F0F0F0F for a packed word q; words 24..26 hold -8 * (sum of
-// the piece's digits of plane i) and word 27 the A_max of the piece's group
-// (fp32 bits).  rec: [K/32][M][28].
-template <int NSUB>
+// R = gemv_rec_words(S) words (28 for S = 3): word i*8 + 2j + h holds digit
+// plane i's bytes for the piece's packed word j, low (h = 0: K offsets 8j +
+// {0, 4, 1, 5}) or high (h = 1: 8j + {2, 6, 3, 7}) nibbles -- the byte order
+// of q & 0x0F0F0F0F and (q >> 4) & 0x0F0F0F0F for a packed word q; words
+// 8S .. 9S-1 hold -8 * (sum of the piece's digits of plane i) and word 9S the
+// A_max of the piece's group (fp32 bits).  rec: [K/32][M][R].
+template <int NSUB, int S>
 __global__ void __launch_bounds__(256) gemv_expand_kernel(const __half* __restrict__ x, int M, int K, int g,
                                                           uint32_t* __restrict__ rec)
 {
+    constexpr int R = gemv_rec_words(S);
     // the matmul that reads the records may launch now and stream its
     // weights; x may come from the previous kernel, and the previous matmul
     // may still read the records this kernel overwrites
@@ -185,34 +189,32 @@ __global__ void __launch_bounds__(256) gemv_expand_kernel(const __half* __restri
 #pragma unroll
     for (int s = 0; s < NSUB; ++s) {
         const int k0 = sp * span + s * kKC + 4 * lane;
-        uint32_t word[3] = {0u, 0u, 0u};
-        int sum[3] = {0, 0, 0};
+        uint32_t word[S];
+        int sum[S];
+#pragma unroll
+        for (int i = 0; i < S; ++i) {
+            word[i] = 0u;
+            sum[i] = 0;
+        }
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            int d1 = 0, d2 = 0, d3 = 0;
             if (am != 0.f) {
-                const float t1 = __fdiv_rn(__fmul_rn(7.49f, v[s][e]), am);
-                const float a1 = rintf(t1);
-                const float t2 = __fmul_rn(__fsub_rn(t1, a1), 14.98f);
-                const float a2 = rintf(t2);
-                const float t3 = __fmul_rn(__fsub_rn(t2, a2), 14.98f);
-                const float a3 = rintf(t3);
-                d1 = static_cast<int>(a1);
-                d2 = static_cast<int>(a2);
-                d3 = static_cast<int>(a3);
+                float t = __fdiv_rn(__fmul_rn(7.49f, v[s][e]), am);
+#pragma unroll
+                for (int i = 0; i < S; ++i) {
+                    const float a = rintf(t);
+                    const int d = static_cast<int>(a);
+                    word[i] |= (static_cast<uint32_t>(d) & 0xFFu) << (8 * e);
+                    sum[i] += d;
+                    if (i + 1 < S) t = __fmul_rn(__fsub_rn(t, a), 14.98f);
+                }
             }
-            word[0] |= (static_cast<uint32_t>(d1) & 0xFFu) << (8 * e);
-            word[1] |= (static_cast<uint32_t>(d2) & 0xFFu) << (8 * e);
-            word[2] |= (static_cast<uint32_t>(d3) & 0xFFu) << (8 * e);
-            sum[0] += d1;
-            sum[1] += d2;
-            sum[2] += d3;
         }
         // lanes 2j and 2j+1 of each 8-lane piece hold K offsets 8j..8j+3 and 8j+4..8j+7
         const int pg = (sp * span + s * kKC) / 32 + (lane >> 3);
-        uint32_t* r = rec + (static_cast<size_t>(pg) * M + m) * kGemvRecWords;
+        uint32_t* r = rec + (static_cast<size_t>(pg) * M + m) * R;
 #pragma unroll
-        for (int i = 0; i < 3; ++i) {
+        for (int i = 0; i < S; ++i) {
             const uint32_t other = __shfl_xor_sync(0xffffffffu, word[i], 1);
             // even lane: [a0 a4 a1 a5] from (mine = a0..a3, other = a4..a7);
             // odd lane:  [a2 a6 a3 a7] from (other = a0..a3, mine = a4..a7)
@@ -224,11 +226,11 @@ __global__ void __launch_bounds__(256) gemv_expand_kernel(const __half* __restri
             t += __shfl_xor_sync(0xffffffffu, t, 4);
             if (k0 < K) {   // a piece lies wholly inside or outside K (K % 32 == 0)
                 r[i * 8 + (lane & 7)] = out;
-                if ((lane & 7) == 0) r[24 + i] = static_cast<uint32_t>(-8 * t);
+                if ((lane & 7) == 0) r[8 * S + i] = static_cast<uint32_t>(-8 * t);
             }
         }
         // a piece lies inside one group (g % 32 == 0)
-        if (k0 < K && (lane & 7) == 0) r[27] = __float_as_uint(am);
+        if (k0 < K && (lane & 7) == 0) r[9 * S] = __float_as_uint(am);
     }
 }
 

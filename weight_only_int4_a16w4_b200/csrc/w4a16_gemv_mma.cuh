@@ -27,7 +27,9 @@
 //    which gemv_expand_kernel writes in exactly this byte order.  Y_i = D -
 //    8 * (sum of the quad's digits), exact in int32; per group the combine
 //    (equations 9-11) Y_i * c_i * A_max * scale is added to an fp32 sum per
-//    (row, column); the three planes of a token are added at the end.
+//    (row, column); the three planes of a token are added at the end.  With
+//    S = 2 or 4 unfold steps the rows are the S planes of each token (S * M
+//    <= 8) and the records carry S planes.
 //  * DEQUANT (m16n8k16, f16 -> f32): a word unpacks to four fp16 pairs of the
 //    exact weights (K offsets (0,1), (2,3), (4,5), (6,7)); the A rows are the
 //    tokens and lane (m, t)'s A registers for word j are x[m][8j .. 8j+7] of
@@ -72,9 +74,11 @@ constexpr int kMgCB = 4;     // 8-column blocks per round (one cell per lane per
 
 template <int VAR, int MR>
 struct MgCfg {
-    static constexpr bool kIsMsd = VAR == kMsd;
+    static constexpr bool kIsMsd = is_msd(VAR);
     static constexpr bool kBf16 = VAR == kDeqBf16;
-    static constexpr int kRows = kIsMsd ? 3 * MR : MR;   // A / D rows in use
+    static constexpr int kS = kIsMsd ? msd_steps(VAR) : 1;   // digit planes per token
+    static constexpr int kRec = gemv_rec_words(kS);          // words per MSD record
+    static constexpr int kRows = kS * MR;                    // A / D rows in use
     // rounds in flight per warp: 4 deep, the CTA alone on its SM (measured:
     // deeper rings beat keeping the next call's CTA resident, except for a
     // dequant call that only ever follows another dequant call)
@@ -85,11 +89,11 @@ struct MgCfg {
     // the most quads (and 32-K pieces) one warp takes
     __host__ __device__ static constexpr int qpw(int npieces) { return (npieces / 4 + kMgWarps - 1) / kMgWarps; }
     __host__ __device__ static constexpr int ppw(int npieces) { return 4 * qpw(npieces); }
-    // one warp's operand: MSD the digit records of its pieces [ppw][M][28
+    // one warp's operand: MSD the digit records of its pieces [ppw][M][kRec
     // words]; DEQUANT its slice of x [M][ppw * 32] fp16
     __host__ __device__ static constexpr int operand_bytes(int M, int npieces)
     {
-        return kIsMsd ? ppw(npieces) * M * kGemvRecWords * 4 : ppw(npieces) * M * 64;
+        return kIsMsd ? ppw(npieces) * M * kRec * 4 : ppw(npieces) * M * 64;
     }
     __host__ __device__ static constexpr int warp_stride(int M, int npieces, int ppg)
     {
@@ -191,7 +195,7 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
     uint8_t* ring = wreg;                                               // [depth][piece][32 cells], swizzled
     uint8_t* sring = wreg + C::kDepth * 4 * 512;                         // [depth][block] 8 fp16 scales
     const uint8_t* opnd = wreg + C::kRing;
-    const uint32_t* rec_w = reinterpret_cast<const uint32_t*>(opnd);    // MSD: [ppw][M][28]
+    const uint32_t* rec_w = reinterpret_cast<const uint32_t*>(opnd);    // MSD: [ppw][M][kRec]
     const __half* xw = reinterpret_cast<const __half*>(opnd);           // DEQUANT: [M][ppw * 32]
 
     // (the host keeps nblk * ctas below 2^31)
@@ -208,17 +212,28 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
     // this lane's A row: MSD (plane, token) = (gl / M, gl % M); DEQUANT token
     // gl.  A lane past the real rows reads a valid row anyway: its MMA rows
     // are never read back.
-    const bool row_ok = gl < (C::kIsMsd ? 3 * M : M);
+    const bool row_ok = gl < C::kS * M;
     int row_m, row_plane;
     if constexpr (C::kIsMsd) {
-        // M is 1 or 2 here
-        row_m = M == 1 ? 0 : (gl & 1);
-        row_plane = min(M == 1 ? gl : (gl >> 1), 2);
+        // the instance's MR fixes M: MR = 1 -> M = 1, MR = 2 -> M = 2,
+        // MR = 4 -> M = 3 or 4
+        if constexpr (MR == 1) {
+            row_m = 0;
+            row_plane = gl;
+        } else if constexpr (MR == 2) {
+            row_m = M == 1 ? 0 : (gl & 1);
+            row_plane = M == 1 ? gl : (gl >> 1);
+        } else {
+            row_m = M == 4 ? (gl & 3) : gl % 3;
+            row_plane = M == 4 ? (gl >> 2) : gl / 3;
+        }
+        row_plane = min(row_plane, C::kS - 1);
     } else {
         row_m = gl < M ? gl : 0;
         row_plane = 0;
     }
-    const float row_c = row_plane == 0 ? kC1 : (row_plane == 1 ? kC2 : kC3);
+    // combine weight 1 / (7.49 * 14.98^plane) of this lane's row
+    const float row_c = (C::kS <= 3 || row_plane < 3) ? (row_plane == 0 ? kC1 : (row_plane == 1 ? kC2 : kC3)) : kC4;
 
     // the next kernel in the stream may start its own weight stream now
     griddep_launch_dependents();
@@ -273,8 +288,8 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
             const __half* sg = reinterpret_cast<const __half*>(sring + slot * kMgCB * 16) + 2 * tl;
             if constexpr (C::kIsMsd) {
                 // lane (row, tl) reads the record of piece 4q + tl
-                const uint32_t* r = rec_w + ((4 * rr + tl) * M + row_m) * kGemvRecWords;
-                int c = static_cast<int>(r[24 + row_plane]);
+                const uint32_t* r = rec_w + ((4 * rr + tl) * M + row_m) * C::kRec;
+                int c = static_cast<int>(r[8 * C::kS + row_plane]);
                 if (!row_ok) c = 0;
                 c += __shfl_xor_sync(0xffffffffu, c, 1);
                 c += __shfl_xor_sync(0xffffffffu, c, 2);
@@ -291,8 +306,8 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
                     }
                 }
                 if (closes) {
-                    // word 27 of a record is the A_max of its group
-                    const float alpha = row_ok ? row_c * __uint_as_float(r[27]) : 0.f;   // rows past 3M: unused
+                    // word 9S of a record is the A_max of its group
+                    const float alpha = row_ok ? row_c * __uint_as_float(r[9 * C::kS]) : 0.f;   // rows past S M: unused
 #pragma unroll
                     for (int k = 0; k < kMgCB; ++k) {
                         if (k >= nbk) break;
@@ -362,10 +377,14 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
 #pragma unroll
                 for (int w = 0; w < kMgWarps; ++w) {
                     const float* rw = r + w * kMgCB * C::kRows * 8;
-                    if constexpr (C::kIsMsd)
-                        s += (rw[m * 8] + rw[(M + m) * 8]) + rw[(2 * M + m) * 8];
-                    else
+                    if constexpr (C::kIsMsd) {
+                        float t = rw[m * 8];
+#pragma unroll
+                        for (int p = 1; p < C::kS; ++p) t += rw[(p * M + m) * 8];
+                        s += t;
+                    } else {
                         s += rw[m * 8];
+                    }
                 }
                 store_elem<C::kBf16>(P.y + static_cast<size_t>(m) * P.N + (bb + k) * 8 + col, s);
             }
@@ -401,8 +420,8 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
     griddep_wait();
     const int npw = pw1 - pw0;
     if constexpr (C::kIsMsd) {
-        const uint8_t* src = reinterpret_cast<const uint8_t*>(P.rec + static_cast<size_t>(pw0) * M * kGemvRecWords);
-        const int nv = npw * M * (kGemvRecWords / 4);
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(P.rec + static_cast<size_t>(pw0) * M * C::kRec);
+        const int nv = npw * M * (C::kRec / 4);
         for (int v = lane; v < nv; v += 32) cp_async16(smem_addr(opnd + v * 16), src + v * 16);
     } else {
         // row m's slice: npw * 4 vectors of 16 bytes

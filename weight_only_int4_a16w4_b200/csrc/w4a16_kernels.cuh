@@ -73,13 +73,23 @@ constexpr int kMaxGroupMsd = 512;        // expand_kernel: at most 16 values per
 // kDeqBf16: the dequant variant with bf16 x, scale and y (the INT4 + BF16
 // pairing of the Humming article, aihirek.info).  Its buffers travel in the
 // same __half-typed fields as bit patterns; the kernels read them as bf16.
-enum Variant { kMsd = 0, kDeq = 1, kDeqBf16 = 2 };
+// kMsd2 / kMsd4: MSD with 2 or 4 unfold steps instead of 3 (the residual
+// recursion of section 4.1 run for S digits; section 7 of the same page notes
+// that the gain varies with the number of MSD unfold steps).
+enum Variant { kMsd = 0, kDeq = 1, kDeqBf16 = 2, kMsd2 = 3, kMsd4 = 4 };
+
+__host__ __device__ constexpr bool is_msd(int v) { return v == kMsd || v == kMsd2 || v == kMsd4; }
+// digits per activation: 3 for the page's algorithm, 2 or 4 for the others
+__host__ __device__ constexpr int msd_steps(int v) { return v == kMsd2 ? 2 : (v == kMsd4 ? 4 : 3); }
 
 // Combine weights of equation 10 (denominators read as 7.49, 7.49*14.98,
 // 7.49*14.98^2: the page prints them with the multiplication sign lost).
 constexpr float kC1 = static_cast<float>(1.0 / 7.49);
 constexpr float kC2 = static_cast<float>(1.0 / (7.49 * 14.98));
 constexpr float kC3 = static_cast<float>(1.0 / (7.49 * 14.98 * 14.98));
+constexpr float kC4 = static_cast<float>(1.0 / (7.49 * 14.98 * 14.98 * 14.98));
+// combine weight of digit plane p (0-based): 1 / (7.49 * 14.98^p)
+__host__ __device__ constexpr float msd_plane_c(int p) { return p == 0 ? kC1 : p == 1 ? kC2 : p == 2 ? kC3 : kC4; }
 
 struct GemmParams {
     int M;          // dense: rows of x; grouped: total tokens T
@@ -129,12 +139,12 @@ struct GemmParams {
 // issuers a group is one chunk, so each issuer owns one buffer.
 template <int VAR, int TT, int ST, int WST, int NCONV, int NEPI, int NISS, bool SEPI>
 struct GemmCfg {
-    static constexpr bool kIsMsd = VAR == kMsd;
+    static constexpr bool kIsMsd = is_msd(VAR);
     static constexpr bool kBf16 = VAR == kDeqBf16;
     static constexpr bool kGroupAcc = kIsMsd || SEPI;      // per-group accumulators + per-group epilogue
-    static constexpr int kVals = kIsMsd ? 3 : 1;           // accumulators per token (Y1..Y3 or y)
+    static constexpr int kVals = kIsMsd ? msd_steps(VAR) : 1;   // accumulators per token (Y1..YS or y)
     static constexpr int kMmaN = kVals * TT;
-    static constexpr int kBBytes = kIsMsd ? 3 * TT * 128 : 2 * TT * 128;   // activation tile per stage
+    static constexpr int kBBytes = kIsMsd ? kVals * TT * 128 : 2 * TT * 128;   // activation tile per stage
     static constexpr int kSBytes = (kIsMsd || SEPI) ? 0 : 1024;            // up to 4 scale rows
     static constexpr int kStage = kBBytes;                                 // activation stage (shared memory)
     // activation stages: on the decode tile the tiles are small and every
@@ -324,9 +334,10 @@ __global__ void repack_kernel(const uint8_t* __restrict__ wl, int K, int N, int 
 //   tmp1 = (7.49f * x) / A_max; A1 = rint(tmp1)
 //   tmp2 = (tmp1 - A1) * 14.98f; A2 = rint(tmp2)
 //   tmp3 = (tmp2 - A2) * 14.98f; A3 = rint(tmp3)
-// A_max == 0 gives zero digits.  Output: xq [3][M][K] int8 (equation 8's
+// and, with S != 3 unfold steps, the same recursion for S digits.
+// A_max == 0 gives zero digits.  Output: xq [S][M][K] int8 (equation 8's
 // A_int, residual-major), amax [G][M] fp32.
-template <int VPL>
+template <int VPL, int S>
 __global__ void __launch_bounds__(256) expand_kernel(const __half* __restrict__ x, int M, int K, int g,
                                                      int8_t* __restrict__ xq, float* __restrict__ amax)
 {
@@ -366,21 +377,20 @@ __global__ void __launch_bounds__(256) expand_kernel(const __half* __restrict__ 
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
 
-    int8_t d1[VPL], d2[VPL], d3[VPL];
+    int8_t d[S][VPL];
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
         if (am == 0.f) {
-            d1[i] = d2[i] = d3[i] = 0;
+#pragma unroll
+            for (int p = 0; p < S; ++p) d[p][i] = 0;
         } else {
-            const float t1 = __fdiv_rn(__fmul_rn(7.49f, v[i]), am);
-            const float a1 = rintf(t1);
-            const float t2 = __fmul_rn(__fsub_rn(t1, a1), 14.98f);
-            const float a2 = rintf(t2);
-            const float t3 = __fmul_rn(__fsub_rn(t2, a2), 14.98f);
-            const float a3 = rintf(t3);
-            d1[i] = static_cast<int8_t>(a1);
-            d2[i] = static_cast<int8_t>(a2);
-            d3[i] = static_cast<int8_t>(a3);
+            float t = __fdiv_rn(__fmul_rn(7.49f, v[i]), am);
+#pragma unroll
+            for (int p = 0; p < S; ++p) {
+                const float a = rintf(t);
+                d[p][i] = static_cast<int8_t>(a);
+                if (p + 1 < S) t = __fmul_rn(__fsub_rn(t, a), 14.98f);
+            }
         }
     }
     const size_t plane = static_cast<size_t>(M) * K;
@@ -388,24 +398,19 @@ __global__ void __launch_bounds__(256) expand_kernel(const __half* __restrict__ 
         // one 4-byte store per plane and 4 digits (4-byte aligned)
 #pragma unroll
         for (int i = 0; i < VPL; i += 4) {
-            uint32_t w1 = 0, w2 = 0, w3 = 0;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                w1 |= (static_cast<uint32_t>(static_cast<uint8_t>(d1[i + e]))) << (8 * e);
-                w2 |= (static_cast<uint32_t>(static_cast<uint8_t>(d2[i + e]))) << (8 * e);
-                w3 |= (static_cast<uint32_t>(static_cast<uint8_t>(d3[i + e]))) << (8 * e);
+            for (int p = 0; p < S; ++p) {
+                uint32_t wd = 0;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) wd |= (static_cast<uint32_t>(static_cast<uint8_t>(d[p][i + e]))) << (8 * e);
+                *reinterpret_cast<uint32_t*>(xq + p * plane + base + i) = wd;
             }
-            *reinterpret_cast<uint32_t*>(xq + base + i) = w1;
-            *reinterpret_cast<uint32_t*>(xq + plane + base + i) = w2;
-            *reinterpret_cast<uint32_t*>(xq + 2 * plane + base + i) = w3;
         }
     } else {
 #pragma unroll
-        for (int i = 0; i < VPL; ++i) {
-            xq[base + i] = d1[i];
-            xq[plane + base + i] = d2[i];
-            xq[2 * plane + base + i] = d3[i];
-        }
+        for (int i = 0; i < VPL; ++i)
+#pragma unroll
+            for (int p = 0; p < S; ++p) xq[p * plane + base + i] = d[p][i];
     }
     if (lane == 0) amax[static_cast<size_t>(gi) * M + m] = am;
 }
@@ -442,9 +447,12 @@ __device__ __forceinline__ bool resolve_tile(const GemmParams& P, int TT, TileCo
     return false;
 }
 
-// Equation 10 with 1/7.49 factored out: Y1 + Y2/14.98 + Y3/14.98^2.
+// Equation 10 with 1/7.49 factored out: Y1 + Y2/14.98 + Y3/14.98^2 (+
+// Y4/14.98^3 with four unfold steps).
 constexpr float kR2 = static_cast<float>(1.0 / 14.98);
 constexpr float kR3 = static_cast<float>(1.0 / (14.98 * 14.98));
+constexpr float kR4 = static_cast<float>(1.0 / (14.98 * 14.98 * 14.98));
+__device__ __forceinline__ constexpr float msd_plane_r(int p) { return p == 1 ? kR2 : (p == 2 ? kR3 : kR4); }
 
 template <int VAR, int TT, int ST, int WST, int NCONV, int NEPI, int NISS, bool SEPI, bool DBG>
 __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, SEPI>::kThreads, 1)
@@ -568,7 +576,7 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
                         mbar_arrive_expect_tx(fb, C::kBBytes);
                         if (C::kIsMsd) {
 #pragma unroll
-                            for (int r = 0; r < 3; ++r)
+                            for (int r = 0; r < C::kVals; ++r)
                                 tma_load_2d(smem_addr(st + r * TT * 128), &tmap, kc * kKC, r * P.M + tc.t0, fb);
                         } else {
                             tma_load_2d(smem_addr(st), &tmap, kc * kKC, tc.t0, fb);
@@ -844,10 +852,9 @@ W4A16_ROLE_UNROLL
                     const float scc = sc * kC1;
 #pragma unroll
                     for (int c = 0; c < TE / 8; ++c) {
-                        uint32_t y1[8], y2[8], y3[8];
-                        tmem_ld8(b_addr + 8 * c, y1);
-                        tmem_ld8(b_addr + TT + 8 * c, y2);
-                        tmem_ld8(b_addr + 2 * TT + 8 * c, y3);
+                        uint32_t yv[C::kVals][8];   // Y1..YS of 8 tokens
+#pragma unroll
+                        for (int p = 0; p < C::kVals; ++p) tmem_ld8(b_addr + p * TT + 8 * c, yv[p]);
                         const float4 a0 = reinterpret_cast<const float4*>(am_slot + tb + 8 * c)[0];
                         const float4 a1 = reinterpret_cast<const float4*>(am_slot + tb + 8 * c)[1];
                         const float am[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
@@ -856,10 +863,10 @@ W4A16_ROLE_UNROLL
                         for (int qq = 0; qq < 8; ++qq) {
                             // exact Y_i as floats (|Y| < 2^22 < 2^24), then equation 10
                             // and equation 11's running sum
-                            const float d1 = __int2float_rn(static_cast<int>(y1[qq]));
-                            const float d2 = __int2float_rn(static_cast<int>(y2[qq]));
-                            const float d3 = __int2float_rn(static_cast<int>(y3[qq]));
-                            const float v = fmaf(d3, kR3, fmaf(d2, kR2, d1));
+                            float v = __int2float_rn(static_cast<int>(yv[0][qq]));
+#pragma unroll
+                            for (int p = 1; p < C::kVals; ++p)
+                                v = fmaf(__int2float_rn(static_cast<int>(yv[p][qq])), msd_plane_r(p), v);
                             acc[8 * c + qq] = fmaf(v, am[qq] * scc, acc[8 * c + qq]);
                         }
                         if (DBG && n_ok && n >= P.dbg_n0 && n < P.dbg_n1) {
@@ -871,9 +878,9 @@ W4A16_ROLE_UNROLL
                                 const int m = tc.t0 + t;
                                 if (t < nt && m >= P.dbg_m0 && m < P.dbg_m1) {
                                     const size_t o = (static_cast<size_t>(m - P.dbg_m0) * P.G + grp) * wn + (n - P.dbg_n0);
-                                    P.dbg_yint[o] = static_cast<int32_t>(y1[qq]);
-                                    P.dbg_yint[plane + o] = static_cast<int32_t>(y2[qq]);
-                                    P.dbg_yint[2 * plane + o] = static_cast<int32_t>(y3[qq]);
+#pragma unroll
+                                    for (int p = 0; p < C::kVals; ++p)
+                                        P.dbg_yint[p * plane + o] = static_cast<int32_t>(yv[p][qq]);
                                     if (n == P.dbg_n0)
                                         P.dbg_amax[static_cast<size_t>(m - P.dbg_m0) * P.G + grp] = am[qq];
                                 }
