@@ -113,6 +113,7 @@ SMALL = [
     (130, 384, 520, 128),                # ragged in every dimension, two MMA issuers
     (8, 1024, 264, 128),                 # the largest warp-MMA GEMV row count
     (2, 4096, 1032, 128),                # a long K with ragged column blocks
+    (1, 1024, 8200, 128),                # the 32-warp GEMV instance (M <= 2, N >= 8192)
 ]
 
 

@@ -274,6 +274,8 @@ MMA_DEQ = [
     (6, 2560, 14344, 512),
     (2, 128, 64, 128),
     (7, 8192, 8, 128),
+    (1, 1024, 8200, 128),                # 32-warp instance (M <= 2, N >= 8192), ragged last block
+    (2, 2048, 16384, 256),               # 32-warp instance, groups over two quads
 ]
 MMA_MSD = [
     (1, 8192, 1024, 128),

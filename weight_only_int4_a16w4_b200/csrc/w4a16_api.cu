@@ -195,28 +195,59 @@ int gemv_mma_rows(int op, int M)
     return std::min(r, cap);
 }
 
-template <int VAR>
-int gemv_mma_smem_var(int MR, int M, int np, int ppg)
+template <int VAR, int NW>
+int gemv_mma_smem_nw(int MR, int M, int np, int ppg)
 {
     // instances exist for S * MR <= 8 only
     constexpr int S = is_msd(VAR) ? msd_steps(VAR) : 1;
     switch (MR) {
-        case 1: return MgCfg<VAR, 1>::smem_bytes(M, np, ppg);
-        case 2: return MgCfg<VAR, 2>::smem_bytes(M, np, ppg);
-        case 4: return MgCfg<VAR, 4 * S <= 8 ? 4 : 1>::smem_bytes(M, np, ppg);
-        default: return MgCfg<VAR, 8 * S <= 8 ? 8 : 1>::smem_bytes(M, np, ppg);
+        case 1: return MgCfg<VAR, 1, NW>::smem_bytes(M, np, ppg);
+        case 2: return MgCfg<VAR, 2, NW>::smem_bytes(M, np, ppg);
+        case 4: return MgCfg<VAR, 4 * S <= 8 ? 4 : 1, NW>::smem_bytes(M, np, ppg);
+        default: return MgCfg<VAR, 8 * S <= 8 ? 8 : 1, NW>::smem_bytes(M, np, ppg);
     }
 }
 
-int gemv_mma_smem(int op, int M, int K, int g)
+template <int VAR>
+int gemv_mma_smem_var(int MR, int NW, int M, int np, int ppg)
+{
+    return NW == 32 ? gemv_mma_smem_nw<VAR, 32>(MR, M, np, ppg) : gemv_mma_smem_nw<VAR, 16>(MR, M, np, ppg);
+}
+
+int gemv_mma_smem_nw_op(int op, int NW, int M, int K, int g)
 {
     const int np = K / 32, ppg = g / 32, MR = gemv_mma_rows(op, M);
     switch (op) {
-        case W4A16_OP_MSD: return gemv_mma_smem_var<kMsd>(MR, M, np, ppg);
-        case W4A16_OP_MSD_2STEP: return gemv_mma_smem_var<kMsd2>(MR, M, np, ppg);
-        case W4A16_OP_MSD_4STEP: return gemv_mma_smem_var<kMsd4>(MR, M, np, ppg);
-        default: return gemv_mma_smem_var<kDeq>(MR, M, np, ppg);
+        case W4A16_OP_MSD: return gemv_mma_smem_var<kMsd>(MR, NW, M, np, ppg);
+        case W4A16_OP_MSD_2STEP: return gemv_mma_smem_var<kMsd2>(MR, NW, M, np, ppg);
+        case W4A16_OP_MSD_4STEP: return gemv_mma_smem_var<kMsd4>(MR, NW, M, np, ppg);
+        default: return gemv_mma_smem_var<kDeq>(MR, NW, M, np, ppg);
     }
+}
+
+// Warps per CTA of the warp-MMA GEMV.  Measured on B200 (us per call, 16 vs
+// 32 warps): dequant at M <= 2 with N >= 8192 gains from 32 warps of one
+// quad-round each (K 4096, N 14336: 17.3 -> 16.3; K = N = 8192: 18.2 ->
+// 16.8); at N = 4096 and for MSD, 16 warps are as fast or faster (MSD
+// K 4096, N 14336: 14.7 vs 15.6); 8 warps lose everywhere.  W4A16_MG_WARPS =
+// 16 | 32 forces one.
+int gemv_mma_warps(int op, int M, int K, int N, int g)
+{
+    static int forced = -1;
+    if (forced < 0) {
+        const char* e = std::getenv("W4A16_MG_WARPS");
+        forced = (e && *e) ? std::atoi(e) : 0;
+    }
+    int nw = 16;
+    if (forced == 16 || forced == 32) nw = forced;
+    else if (!is_msd_op(op) && M <= 2 && N >= 8192) nw = 32;
+    if (nw == 32 && gemv_mma_smem_nw_op(op, 32, M, K, g) > kMaxSmemOptin) nw = 16;
+    return nw;
+}
+
+int gemv_mma_smem(int op, int M, int K, int N, int g)
+{
+    return gemv_mma_smem_nw_op(op, gemv_mma_warps(op, M, K, N, g), M, K, g);
 }
 
 // The kernel of a dense call with a handful of rows.  Measured on B200
@@ -248,7 +279,7 @@ int small_kernel(int op, int M, int K, int N, int g, int E)
     if (E != 1 || M < 1) return kSmallNone;
     const bool mma_ok = g % 128 == 0 && M <= gemv_mma_max_m(op) &&
                         static_cast<long long>(N / 8) * sm_count() < (1ll << 31) &&
-                        gemv_mma_smem(op, M, K, g) <= kMaxSmemOptin;
+                        gemv_mma_smem(op, M, K, N, g) <= kMaxSmemOptin;
     // (the CUDA-core GEMV is built for fp16 dequant and three-step MSD only)
     const bool cuda_ok = (op == W4A16_OP_DEQUANT || op == W4A16_OP_MSD) && M <= 4 &&
                          static_cast<long long>(M) * K <= kGemvMaxMK;
@@ -514,13 +545,11 @@ w4a16_status launch_gemv_mr(const GemvParams& P, cudaStream_t stream)
     return W4A16_OK;
 }
 
-template <int VAR, int MR>
-w4a16_status launch_gemv_mma_mr(const GemvParams& P, cudaStream_t stream)
+template <int VAR, int MR, int NW>
+w4a16_status launch_gemv_mma_nw(const GemvParams& P, cudaStream_t stream)
 {
-    auto kern = gemv_mma_kernel<VAR, MR>;
-    const int op = VAR == kMsd ? W4A16_OP_MSD : VAR == kMsd2 ? W4A16_OP_MSD_2STEP
-                 : VAR == kMsd4 ? W4A16_OP_MSD_4STEP : W4A16_OP_DEQUANT;
-    const int smem = gemv_mma_smem(op, P.M, P.K, P.g);
+    auto kern = gemv_mma_kernel<VAR, MR, NW>;
+    const int smem = MgCfg<VAR, MR, NW>::smem_bytes(P.M, P.K / 32, P.g / 32);
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
@@ -530,7 +559,7 @@ w4a16_status launch_gemv_mma_mr(const GemvParams& P, cudaStream_t stream)
     if (smem > kMaxSmemOptin) return W4A16_ERR_UNSUPPORTED;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(P.ctas), 1, 1);
-    cfg.blockDim = dim3(kMgThreads, 1, 1);
+    cfg.blockDim = dim3(NW * 32, 1, 1);
     cfg.dynamicSmemBytes = static_cast<size_t>(smem);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -543,6 +572,15 @@ w4a16_status launch_gemv_mma_mr(const GemvParams& P, cudaStream_t stream)
         return W4A16_ERR_CUDA;
     }
     return W4A16_OK;
+}
+
+template <int VAR, int MR>
+w4a16_status launch_gemv_mma_mr(const GemvParams& P, cudaStream_t stream)
+{
+    const int op = VAR == kMsd ? W4A16_OP_MSD : VAR == kMsd2 ? W4A16_OP_MSD_2STEP
+                 : VAR == kMsd4 ? W4A16_OP_MSD_4STEP : W4A16_OP_DEQUANT;
+    if (gemv_mma_warps(op, P.M, P.K, P.N, P.g) == 32) return launch_gemv_mma_nw<VAR, MR, 32>(P, stream);
+    return launch_gemv_mma_nw<VAR, MR, 16>(P, stream);
 }
 
 template <int NSUB, int S>

@@ -143,6 +143,55 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p)
 // of q & 0x0F0F0F0F and (q >> 4) & 0x0F0F0F0F for a packed word q; words
 // 8S .. 9S-1 hold -8 * (sum of the piece's digits of plane i) and word 9S the
 // A_max of the piece's group (fp32 bits).  rec: [K/32][M][R].
+// Digits and record of one 128-K sub-chunk of one row (steps 2-8 in IEEE
+// binary32, the literal operation order): lane l holds the sub-chunk's values
+// 4l .. 4l+3 in v and am, the A_max of their group; every lane takes part in
+// the shuffles, and lanes with `store` write the record of their 32-K piece
+// (lane / 8) at r.
+template <int S>
+__device__ __forceinline__ void msd_subchunk_record(const float (&v)[4], float am, int lane, uint32_t* r, bool store)
+{
+    uint32_t word[S];
+    int sum[S];
+#pragma unroll
+    for (int i = 0; i < S; ++i) {
+        word[i] = 0u;
+        sum[i] = 0;
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        if (am != 0.f) {
+            float t = __fdiv_rn(__fmul_rn(7.49f, v[e]), am);
+#pragma unroll
+            for (int i = 0; i < S; ++i) {
+                const float a = rintf(t);
+                const int d = static_cast<int>(a);
+                word[i] |= (static_cast<uint32_t>(d) & 0xFFu) << (8 * e);
+                sum[i] += d;
+                if (i + 1 < S) t = __fmul_rn(__fsub_rn(t, a), 14.98f);
+            }
+        }
+    }
+    // lanes 2j and 2j+1 of each 8-lane piece hold K offsets 8j..8j+3 and 8j+4..8j+7
+#pragma unroll
+    for (int i = 0; i < S; ++i) {
+        const uint32_t other = __shfl_xor_sync(0xffffffffu, word[i], 1);
+        // even lane: [a0 a4 a1 a5] from (mine = a0..a3, other = a4..a7);
+        // odd lane:  [a2 a6 a3 a7] from (other = a0..a3, mine = a4..a7)
+        const uint32_t out = (lane & 1) ? __byte_perm(other, word[i], 0x7362) : __byte_perm(word[i], other, 0x5140);
+        int t = sum[i];
+        t += __shfl_xor_sync(0xffffffffu, t, 1);
+        t += __shfl_xor_sync(0xffffffffu, t, 2);
+        t += __shfl_xor_sync(0xffffffffu, t, 4);
+        if (store) {
+            r[i * 8 + (lane & 7)] = out;
+            if ((lane & 7) == 0) r[8 * S + i] = static_cast<uint32_t>(-8 * t);
+        }
+    }
+    // a piece lies inside one group (g % 32 == 0)
+    if (store && (lane & 7) == 0) r[9 * S] = __float_as_uint(am);
+}
+
 template <int NSUB, int S>
 __global__ void __launch_bounds__(256) gemv_expand_kernel(const __half* __restrict__ x, int M, int K, int g,
                                                           uint32_t* __restrict__ rec)
@@ -189,48 +238,9 @@ __global__ void __launch_bounds__(256) gemv_expand_kernel(const __half* __restri
 #pragma unroll
     for (int s = 0; s < NSUB; ++s) {
         const int k0 = sp * span + s * kKC + 4 * lane;
-        uint32_t word[S];
-        int sum[S];
-#pragma unroll
-        for (int i = 0; i < S; ++i) {
-            word[i] = 0u;
-            sum[i] = 0;
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            if (am != 0.f) {
-                float t = __fdiv_rn(__fmul_rn(7.49f, v[s][e]), am);
-#pragma unroll
-                for (int i = 0; i < S; ++i) {
-                    const float a = rintf(t);
-                    const int d = static_cast<int>(a);
-                    word[i] |= (static_cast<uint32_t>(d) & 0xFFu) << (8 * e);
-                    sum[i] += d;
-                    if (i + 1 < S) t = __fmul_rn(__fsub_rn(t, a), 14.98f);
-                }
-            }
-        }
-        // lanes 2j and 2j+1 of each 8-lane piece hold K offsets 8j..8j+3 and 8j+4..8j+7
         const int pg = (sp * span + s * kKC) / 32 + (lane >> 3);
-        uint32_t* r = rec + (static_cast<size_t>(pg) * M + m) * R;
-#pragma unroll
-        for (int i = 0; i < S; ++i) {
-            const uint32_t other = __shfl_xor_sync(0xffffffffu, word[i], 1);
-            // even lane: [a0 a4 a1 a5] from (mine = a0..a3, other = a4..a7);
-            // odd lane:  [a2 a6 a3 a7] from (other = a0..a3, mine = a4..a7)
-            const uint32_t out =
-                (lane & 1) ? __byte_perm(other, word[i], 0x7362) : __byte_perm(word[i], other, 0x5140);
-            int t = sum[i];
-            t += __shfl_xor_sync(0xffffffffu, t, 1);
-            t += __shfl_xor_sync(0xffffffffu, t, 2);
-            t += __shfl_xor_sync(0xffffffffu, t, 4);
-            if (k0 < K) {   // a piece lies wholly inside or outside K (K % 32 == 0)
-                r[i * 8 + (lane & 7)] = out;
-                if ((lane & 7) == 0) r[8 * S + i] = static_cast<uint32_t>(-8 * t);
-            }
-        }
-        // a piece lies inside one group (g % 32 == 0)
-        if (k0 < K && (lane & 7) == 0) r[9 * S] = __float_as_uint(am);
+        // a piece lies wholly inside or outside K (K % 32 == 0)
+        msd_subchunk_record<S>(v[s], am, lane, rec + (static_cast<size_t>(pg) * M + m) * R, k0 < K);
     }
 }
 

@@ -52,7 +52,8 @@
 // (programmatic dependent launch), so the weight stream of a call overlaps
 // the tail of the previous one.  The weights hold no registers in flight, so 16 warps of
 // at most 64 registers keep enough loads outstanding (the memory system
-// wants many warps with a few loads each).
+// wants many warps with a few loads each).  A 32-warp instance (two rounds in
+// flight per warp, one CTA per SM) serves wide dequant calls.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -67,13 +68,14 @@
 
 namespace w4a16 {
 
-constexpr int kMgWarps = 16;
-constexpr int kMgThreads = kMgWarps * 32;
+constexpr int kMgWarps = 16;                 // warps of the default instance (NW)
 constexpr int kMgCB = 4;     // 8-column blocks per round (one cell per lane per piece)
 
 
-template <int VAR, int MR>
+template <int VAR, int MR, int NW = kMgWarps>
 struct MgCfg {
+    static constexpr int kWarps = NW;
+    static constexpr int kThreads = NW * 32;
     static constexpr bool kIsMsd = is_msd(VAR);
     static constexpr bool kBf16 = VAR == kDeqBf16;
     static constexpr int kS = kIsMsd ? msd_steps(VAR) : 1;   // digit planes per token
@@ -82,12 +84,13 @@ struct MgCfg {
     // rounds in flight per warp: 4 deep, the CTA alone on its SM (measured:
     // deeper rings beat keeping the next call's CTA resident, except for a
     // dequant call that only ever follows another dequant call)
-    static constexpr int kDepth = 4;
+    static constexpr int kDepth = NW >= 32 ? 2 : 4;
     static constexpr int kRing = kDepth * 4 * 512 + kDepth * kMgCB * 16;   // weight cells + scales, per warp
     static_assert(kRows <= 8, "rows must fit the lower half of the m16 tile");
-    static constexpr int kRed = kMgWarps * kMgCB * kRows * 8 * 4;   // [warp][block][row][column] fp32
+    static constexpr int kRed = NW * kMgCB * kRows * 8 * 4;   // [warp][block][row][column] fp32
+    static_assert(kMgCB * MR * 8 <= NW * 32, "the final sum needs a thread per (block, row, column)");
     // the most quads (and 32-K pieces) one warp takes
-    __host__ __device__ static constexpr int qpw(int npieces) { return (npieces / 4 + kMgWarps - 1) / kMgWarps; }
+    __host__ __device__ static constexpr int qpw(int npieces) { return (npieces / 4 + NW - 1) / NW; }
     __host__ __device__ static constexpr int ppw(int npieces) { return 4 * qpw(npieces); }
     // one warp's operand: MSD the digit records of its pieces [ppw][M][kRec
     // words]; DEQUANT its slice of x [M][ppw * 32] fp16
@@ -101,7 +104,7 @@ struct MgCfg {
     }
     __host__ __device__ static constexpr int smem_bytes(int M, int npieces, int ppg)
     {
-        return kRed + kMgWarps * warp_stride(M, npieces, ppg);
+        return kRed + NW * warp_stride(M, npieces, ppg);
     }
 };
 
@@ -180,10 +183,10 @@ __device__ __forceinline__ void unpack_exact_f16(uint32_t q, uint32_t (&p)[4])
     p[3] = *reinterpret_cast<const uint32_t*>(&w3);
 }
 
-template <int VAR, int MR>
-__global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_constant__ GemvParams P)
+template <int VAR, int MR, int NW>
+__global__ void __launch_bounds__(NW * 32, NW >= 32 ? 1 : 2) gemv_mma_kernel(const __grid_constant__ GemvParams P)
 {
-    using C = MgCfg<VAR, MR>;
+    using C = MgCfg<VAR, MR, NW>;
     extern __shared__ __align__(16) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gl = lane >> 2, tl = lane & 3;   // fragment row / column group of this lane
@@ -202,7 +205,7 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
     const int b0 = static_cast<int>((blockIdx.x * static_cast<unsigned>(P.nblk)) / static_cast<unsigned>(P.ctas));
     const int b1 = static_cast<int>(((blockIdx.x + 1) * static_cast<unsigned>(P.nblk)) / static_cast<unsigned>(P.ctas));
     const int nq = P.npieces / 4;
-    const int qw0 = (warp * nq) / kMgWarps, qw1 = ((warp + 1) * nq) / kMgWarps;
+    const int qw0 = (warp * nq) / NW, qw1 = ((warp + 1) * nq) / NW;
     const int pw0 = 4 * qw0, pw1 = 4 * qw1;
     const int rpb = C::qpw(P.npieces);                  // rounds per block-group (same for every warp)
     const int gw0 = qw0 / qpg, qpos0 = qw0 - gw0 * qpg;  // the warp's first group, its quads before qw0
@@ -375,7 +378,7 @@ __global__ void __launch_bounds__(kMgThreads, 2) gemv_mma_kernel(const __grid_co
                 const float* r = red + (k * C::kRows) * 8 + col;
                 float s = 0.f;
 #pragma unroll
-                for (int w = 0; w < kMgWarps; ++w) {
+                for (int w = 0; w < NW; ++w) {
                     const float* rw = r + w * kMgCB * C::kRows * 8;
                     if constexpr (C::kIsMsd) {
                         float t = rw[m * 8];
