@@ -606,8 +606,13 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
         // that reconverges after every MMA roughly doubles the issue cost of
         // each one.
         if (q < issuers && lane == 0) {
-            constexpr uint32_t idesc = C::kIsMsd ? idesc_s8_s32(C::kMmaN)
-                                                 : (C::kBf16 ? idesc_bf16_f32(C::kMmaN) : idesc_f16_f32(C::kMmaN));
+            // dequant: a tile's MMAs cover only its tokens, rounded up to the
+            // MMA's N step of 16 (the ragged last tile of an expert segment
+            // then costs a fraction of a full one); the rows past them are
+            // never read back.  MSD stacks its digit planes along N: full N.
+            const int n_eff = C::kIsMsd ? C::kMmaN : min(C::kMmaN, ((tc.t_end - tc.t0 + 15) / 16) * 16);
+            const uint32_t idesc = C::kIsMsd ? idesc_s8_s32(C::kMmaN)
+                                             : (C::kBf16 ? idesc_bf16_f32(n_eff) : idesc_f16_f32(n_eff));
             constexpr int kSteps = C::kIsMsd ? 4 : 8;         // MMA K steps per 128-deep chunk
             constexpr int kStepK = kKC / kSteps;
             // group bookkeeping without divisions in the step loop: K steps
