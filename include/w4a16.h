@@ -245,7 +245,10 @@ w4a16_status w4a16_moe_workspace_size(int op, int T, int topk, int K, int N, int
                                       int E, size_t* bytes);
 
 /* The routed grouped form end to end: align, gather, grouped matmul,
- * combine, on one stream, no host synchronisation.  x fp16 [T][K], y fp16
+ * combine, on one stream, no host synchronisation.  With topk == 1 the
+ * combine is fused into the grouped matmul's stores (each row written at its
+ * token times the gate weight; a token whose id lies outside [0, E) gets a
+ * zero row).  x fp16 [T][K], y fp16
  * [T][N] (both bf16 for W4A16_OP_DEQUANT_BF16); w_packed / scale as
  * w4a16_grouped_matmul; topk_ids, topk_weights device [T][topk]. */
 w4a16_status w4a16_moe_matmul(int op, const void* x, const int32_t* topk_ids,

@@ -197,13 +197,15 @@ def test_grouped_bf16_matches_oracle(cuda_lib, T, K, N, g, E):
     assert_bf16_close(run_grouped(w4, c, dev), ref, S, K, g, f"grouped bf16 T{T} E{E}")
 
 
-def test_moe_matmul_bf16_end_to_end(cuda_lib):
+@pytest.mark.parametrize("topk", [1, 2])
+def test_moe_matmul_bf16_end_to_end(cuda_lib, topk):
     """Router entries grouped, gathered, multiplied and added back with the
     gate weights, all in bf16: each row's y is rounded to bf16 once before the
-    fp32 gate-weighted sum, so the bar adds u times the rows' weighted sizes."""
+    fp32 gate-weighted sum (topk = 1: the weight is applied in the matmul's
+    stores, one rounding), so the bar adds u times the rows' weighted sizes."""
     w4 = cuda_lib
     torch = _t()
-    T, topk, E, K, N, g = 37, 2, 5, 256, 136, 64
+    T, E, K, N, g = 37, 5, 256, 136, 64
     rng = np.random.default_rng(5)
     c = make_case(T, K, N, g, seed=91, E=E, grouped=False, act="bf16")
     ids = rng.integers(0, E, (T, topk)).astype(np.int32)

@@ -97,6 +97,8 @@ def test_moe_combine_within_one_ulp(w4, T, topk, N):
     (37, 2, 5, 256, 264, 64, False),
     (150, 2, 8, 512, 136, 128, True),
     (9, 1, 3, 1024, 520, 256, False),
+    (200, 1, 4, 256, 264, 64, True),       # one expert per token: fused un-permute, dropped ids give zero rows
+    (300, 1, 8, 512, 136, 128, False),     # fused un-permute on the large tiles, ragged segments
 ])
 def test_moe_matmul_end_to_end(w4, op, T, topk, E, K, N, g, invalid):
     import torch

@@ -890,9 +890,13 @@ w4a16_status w4a16_msd_debug_yint(const void* x, const void* w_packed, int M, in
                                       workspace_bytes, stream);
 }
 
-w4a16_status w4a16_grouped_matmul(int op, const void* x, const void* const* w_packed, const void* const* scale,
-                                  const int32_t* offsets, int E, int T, int K, int N, int group_size, void* y,
-                                  void* workspace, size_t workspace_bytes, w4a16_stream_t stream)
+namespace {
+// The grouped matmul; row_dst / row_w (routed form, one expert per token)
+// store row r at y row row_dst[r] times row_w[row_dst[r]] (nullptr: row r).
+w4a16_status grouped_impl(int op, const void* x, const void* const* w_packed, const void* const* scale,
+                          const int32_t* offsets, int E, int T, int K, int N, int group_size, void* y,
+                          void* workspace, size_t workspace_bytes, const int32_t* row_dst, const float* row_w,
+                          w4a16_stream_t stream)
 {
     if (!op_ok(op)) return W4A16_ERR_INVALID_ARG;
     if (E < 1 || E > kMaxExperts) return W4A16_ERR_INVALID_ARG;
@@ -920,6 +924,8 @@ w4a16_status w4a16_grouped_matmul(int op, const void* x, const void* const* w_pa
         P.scale[e] = static_cast<const __half*>(scale[e]);
     }
     P.y = static_cast<__half*>(y);
+    P.row_dst = row_dst;
+    P.row_w = row_w;
     CUtensorMap map;
     if (is_msd_op(op)) {
         int8_t* xq = reinterpret_cast<int8_t*>(wsb + L.xq);
@@ -934,6 +940,15 @@ w4a16_status w4a16_grouped_matmul(int op, const void* x, const void* const* w_pa
     }
     dim3 grid(s.n_tiles, 1, s.t_slots);
     return launch_for(op, s.TT, map, P, grid, cs);
+}
+}  // namespace
+
+w4a16_status w4a16_grouped_matmul(int op, const void* x, const void* const* w_packed, const void* const* scale,
+                                  const int32_t* offsets, int E, int T, int K, int N, int group_size, void* y,
+                                  void* workspace, size_t workspace_bytes, w4a16_stream_t stream)
+{
+    return grouped_impl(op, x, w_packed, scale, offsets, E, T, K, N, group_size, y, workspace, workspace_bytes,
+                        nullptr, nullptr, stream);
 }
 
 w4a16_status w4a16_moe_align(const int32_t* topk_ids, int T, int topk, int E, int32_t* offsets,
@@ -1050,6 +1065,17 @@ w4a16_status w4a16_moe_matmul(int op, const void* x, const int32_t* topk_ids, co
     if ((st = w4a16_moe_align(topk_ids, T, topk, E, offsets, sorted, inv, workspace, L.grouped, stream)) != W4A16_OK)
         return st;
     if ((st = w4a16_moe_gather(x, sorted, rows, K, wsb + L.xs, stream)) != W4A16_OK) return st;
+    if (topk == 1) {
+        // one expert per token: the matmul stores each row at its token, times
+        // the gate weight (the un-permute fused into its stores); tokens whose
+        // id took no row get zeros
+        if ((st = grouped_impl(op, wsb + L.xs, w_packed, scale, offsets, E, rows, K, N, group_size, y, workspace,
+                               L.grouped, sorted, topk_weights, stream)) != W4A16_OK)
+            return st;
+        moe_zero_unrouted_kernel<<<cdiv(T, 8), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+            inv, T, N / 8, static_cast<uint4*>(y));
+        return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+    }
     if ((st = w4a16_grouped_matmul(op, wsb + L.xs, w_packed, scale, offsets, E, rows, K, N, group_size, wsb + L.ys,
                                    workspace, L.grouped, stream)) != W4A16_OK)
         return st;

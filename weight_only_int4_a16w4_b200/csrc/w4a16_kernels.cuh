@@ -105,6 +105,11 @@ struct GemmParams {
     const uint8_t* w[kMaxExperts];          // packed weights per expert
     const __half* scale[kMaxExperts];       // [G][N] per expert
     __half* y;                              // [M][N]
+    // routed form with one expert per token: row r of the grouped result goes
+    // to y row row_dst[r], times the gate weight row_w[row_dst[r]]; nullptr:
+    // row r to row r
+    const int32_t* row_dst;
+    const float* row_w;
     const float* amax;                      // MSD: [G][M]
     uint32_t* status;
     unsigned long long timeout_ns;
@@ -272,6 +277,20 @@ __device__ __forceinline__ void store_elem(__half* p, float v)
 {
     if constexpr (BF) *reinterpret_cast<__nv_bfloat16*>(p) = __float2bfloat16_rn(v);
     else *p = __float2half_rn(v);
+}
+
+// Row r of a tile's result, column n: stored at its own row, or (routed form,
+// one expert per token) at its token's row times the token's gate weight.
+
+template <bool BF>
+__device__ __forceinline__ void store_row(const GemmParams& P, int r, int n, float v)
+{
+    if (P.row_dst == nullptr) {
+        store_elem<BF>(P.y + static_cast<size_t>(r) * P.N + n, v);
+        return;
+    }
+    const int dst = __ldg(P.row_dst + r);
+    if (dst >= 0) store_elem<BF>(P.y + static_cast<size_t>(dst) * P.N + n, v * __ldg(P.row_w + dst));
 }
 
 // Eight int4 weights of one packed word -> two words of four signed int8 in
@@ -795,6 +814,31 @@ W4A16_ROLE_UNROLL
         constexpr int TE = C::kTokPerEpi;
         const int tb = C::kEpiRR ? 0 : eg * TE;                 // first token of this group
         const uint32_t t_addr = tmem + (lane_base << 16);
+        // routed form (one expert per token): the tile's row -> (token, gate
+        // weight) map, staged once per warp in the warp's own A_max ring (not
+        // in use by then) so that the stores do not chase two dependent global
+        // loads per element: [TT] tokens, then [TT] weights
+        auto stage_map = [&]() {
+            float* mp = amax_sm + (warp - C::kEpiWarp0) * 2 * TT;
+            __syncwarp();
+            for (int t = lane; t < TT; t += 32) {
+                int d = -1;
+                float wv = 0.f;
+                if (t < nt) {
+                    d = __ldg(P.row_dst + tc.t0 + t);
+                    if (d >= 0) wv = __ldg(P.row_w + d);
+                }
+                mp[t] = __int_as_float(d);
+                mp[TT + t] = wv;
+            }
+            __syncwarp();
+        };
+        // token t of the tile, column n, through the staged map
+        auto store_mapped = [&](int t, float v) {
+            const float* mp = amax_sm + (warp - C::kEpiWarp0) * 2 * TT;
+            const int d = __float_as_int(mp[t]);
+            if (d >= 0) store_elem<C::kBf16>(P.y + static_cast<size_t>(d) * P.N + n, v * mp[TT + t]);
+        };
         float acc[TE];
 #pragma unroll
         for (int t = 0; t < TE; ++t) acc[t] = 0.f;
@@ -919,7 +963,12 @@ W4A16_ROLE_UNROLL
 #pragma unroll
                         for (int t = 0; t < TE; ++t) acc[t] += rr_part[((e2 - 1) * TT + t) * kBN + r];
             }
-            if (ok && P.splits == 1 && P.write_y && n_ok && (!C::kEpiRR || eg == 0)) {
+            if (P.row_dst != nullptr) {
+                stage_map();
+                if (ok && P.write_y && n_ok)
+                    for (int t = 0; t < TE; ++t)
+                        if (tb + t < nt) store_mapped(tb + t, acc[t]);
+            } else if (ok && P.splits == 1 && P.write_y && n_ok && (!C::kEpiRR || eg == 0)) {
 #pragma unroll
                 for (int t = 0; t < TE; ++t)
                     if (tb + t < nt) store_elem<C::kBf16>(P.y + static_cast<size_t>(tc.t0 + tb + t) * P.N + n, acc[t]);
@@ -928,6 +977,7 @@ W4A16_ROLE_UNROLL
             // one accumulator over all of K per issuer (scales applied by the
             // converter); issuers with no chunk left theirs unwritten
             griddep_wait();
+            if (P.row_dst != nullptr) stage_map();
             const int nacc = min(issuers, nchunks);
             ok = nchunks > 0;
             for (int q = 0; q < nacc && ok; ++q)
@@ -955,8 +1005,13 @@ W4A16_ROLE_UNROLL
                     if (P.write_y && n_ok) {
 #pragma unroll
                         for (int k = 0; k < 16; ++k)
-                            if (tb + 16 * c + k < nt)
-                                store_elem<C::kBf16>(P.y + static_cast<size_t>(tc.t0 + tb + 16 * c + k) * P.N + n, v[k]);
+                            if (tb + 16 * c + k < nt) {
+                                if (P.row_dst == nullptr)
+                                    store_elem<C::kBf16>(P.y + static_cast<size_t>(tc.t0 + tb + 16 * c + k) * P.N + n,
+                                                         v[k]);
+                                else
+                                    store_mapped(tb + 16 * c + k, v[k]);
+                            }
                     }
                 }
                 tc_fence_before();
@@ -1004,7 +1059,7 @@ W4A16_ROLE_UNROLL
                 if (t >= nt || nn >= P.N) continue;
                 float sum = 0.f;
                 for (int sp = 0; sp < S; ++sp) sum += red[sp * per + el];
-                store_elem<C::kBf16>(P.y + static_cast<size_t>(tc.t0 + t) * P.N + nn, sum);
+                store_row<C::kBf16>(P, tc.t0 + t, nn, sum);
             }
         }
         if (warp == C::kEpiWarp0 && lane == 0) W4A16_TRACE_AT(55);

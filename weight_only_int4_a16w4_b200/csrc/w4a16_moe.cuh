@@ -195,4 +195,16 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(const __half* __restri
     }
 }
 
+// Routed form with one expert per token, whose matmul stores each row at its
+// token directly: a token whose entry took no row (an id outside [0, E)) gets
+// a zero row here.  A warp per token.
+__global__ void __launch_bounds__(256) moe_zero_unrouted_kernel(const int32_t* __restrict__ inv_pos, int T, int nv,
+                                                                uint4* __restrict__ y)
+{
+    const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (t >= T || inv_pos[t] >= 0) return;
+    uint4* row = y + static_cast<size_t>(t) * nv;
+    for (int v = lane; v < nv; v += 32) row[v] = make_uint4(0u, 0u, 0u, 0u);
+}
+
 }  // namespace w4a16
