@@ -23,6 +23,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -143,7 +144,9 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        # the raw samples: W4A16_CLOCKS_DIR if set, else the system temp dir
+        out = os.environ.get("W4A16_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(out, f"w4a16_clocks_rank{gpu_index}_{os.getpid()}.csv")
 
     def start(self):
         try:
@@ -402,6 +405,7 @@ def run_e2e(args, G, torch, w4, stream, device):
     wl = G.wl
     x_host = torch.from_numpy(G.c.x).pin_memory()
     y_host = {op: torch.empty((wl.M, wl.N), dtype=torch.float16).pin_memory() for op in (w4.OP_MSD, w4.OP_DEQUANT)}
+    y_np = {op: t.numpy() for op, t in y_host.items()}     # host views of the pinned results
     x_dev = torch.empty_like(G.x[0])
     steps = max(3, min(args.e2e_steps, args.steps))
 
@@ -421,7 +425,7 @@ def run_e2e(args, G, torch, w4, stream, device):
                     e0.record(stream)
                 submit(s)
                 stream.synchronize()          # the host reads both results every step
-                _ = float(y_host[w4.OP_MSD][0, 0]) + float(y_host[w4.OP_DEQUANT][0, 0])
+                _ = float(y_np[w4.OP_MSD][0, 0]) + float(y_np[w4.OP_DEQUANT][0, 0])
             e1 = torch.cuda.Event(enable_timing=True)
             e1.record(stream)
         stream.synchronize()
