@@ -140,3 +140,29 @@ def test_workload_msd_steps_sampled(cuda_lib, S, name):
                      f"{name} S={S}")
     m0 = max(0, c.M - 16)
     check_yint_steps(w4, S, c, dev, m0, c.M, c.N - 40, c.N)
+
+
+@pytest.mark.parametrize("S,topk", [(2, 1), (4, 2)])
+def test_routed_msd_steps(cuda_lib, S, topk):
+    """The routed form (grouping, gather, grouped matmul, un-permute) with the
+    step variants: per token the gate-weighted sum over its experts of the
+    oracle's S-step rows."""
+    w4 = cuda_lib
+    torch = _t()
+    T, E, K, N, g = 45, 3, 256, 136, 64
+    rng = np.random.default_rng(100 + S)
+    c = make_case(T, K, N, g, seed=300 + S, E=E, grouped=False)
+    ids = rng.integers(0, E, (T, topk)).astype(np.int32)
+    wts = rng.uniform(0, 1, (T, topk)).astype(np.float32)
+    dev = upload(w4, c)
+    ws = torch.zeros(w4.w4a16_moe_workspace_size(OPS[S], T, topk, K, N, g, E), dtype=torch.uint8, device="cuda")
+    y = torch.full((T, N), float("nan"), dtype=torch.float16, device="cuda")
+    w4.w4a16_moe_matmul(OPS[S], dev["x"], torch.from_numpy(ids).cuda(), torch.from_numpy(wts).cuda(), dev["wp"],
+                        dev["scale"], E, T, topk, K, N, g, y, ws)
+    assert w4.w4a16_read_status(ws) == 0
+    rows = [oracle.msd_steps(c.x, c.wp[e], c.scale[e], g, S) for e in range(E)]
+    ref = np.zeros((T, N))
+    for t in range(T):
+        for j in range(topk):
+            ref[t] += float(wts[t, j]) * rows[int(ids[t, j])][t]
+    assert_msd_close(y.cpu().numpy().astype(np.float64), ref, f"routed S={S} topk={topk}")
