@@ -56,6 +56,28 @@ bool group_ok(int g)
 
 // ---------------------------------------------------------------- device facts
 
+// cudaFuncSetAttribute acts on the current device, so a kernel's attributes
+// are set once per (kernel instance, device); each launcher keeps one of
+// these.  `init` runs with the device current and returns its CUDA status.
+struct PerDeviceInit {
+    std::mutex mu;
+    std::atomic<bool> done[64] = {};
+    cudaError_t err[64] = {};
+    template <typename Fn>
+    cudaError_t get(Fn&& init)
+    {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+        if (done[dev].load(std::memory_order_acquire)) return err[dev];
+        std::lock_guard<std::mutex> lock(mu);
+        if (!done[dev].load(std::memory_order_relaxed)) {
+            err[dev] = init();
+            done[dev].store(true, std::memory_order_release);
+        }
+        return err[dev];
+    }
+};
+
 int sm_count()
 {
     static std::mutex mu;
@@ -349,14 +371,16 @@ w4a16_status launch_gemm(const CUtensorMap& map, const GemmParams& P, dim3 grid,
 {
     using C = GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, SEPI>;
     auto kern = gemm_kernel<VAR, TT, ST, WST, NCONV, NEPI, NISS, SEPI, DBG>;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [&] {
-        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-        if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    static PerDeviceInit kattr;
+    const cudaError_t attr_err = kattr.get([&] {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        return e;
     });
-    if (attr_err != cudaSuccess) return W4A16_ERR_CUDA;
+    if (attr_err != cudaSuccess) {
+        (void)cudaGetLastError();
+        return W4A16_ERR_CUDA;
+    }
     // split-K reduces through the decode tile's own partial buffer
     if (P.splits > 1 && (C::kRedBytes == 0 || P.splits > 16)) return W4A16_ERR_UNSUPPORTED;
     if (P.issuers < 1 || P.issuers > NISS || ST % P.issuers != 0) return W4A16_ERR_UNSUPPORTED;
@@ -521,12 +545,14 @@ w4a16_status launch_gemv_mr(const GemvParams& P, cudaStream_t stream)
     using C = GemvCfg<VAR, MR>;
     auto kern = gemv_kernel<VAR, MR>;
     const int smem = C::smem_bytes(P.M, P.K);
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [&] {
-        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmemOptin);
-    });
-    if (attr_err != cudaSuccess) return W4A16_ERR_CUDA;
+    static PerDeviceInit kattr;
+    const auto set_smem = [&] {
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmemOptin);
+    };
+    if (kattr.get(set_smem) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return W4A16_ERR_CUDA;
+    }
     if (smem > kMaxSmemOptin) return W4A16_ERR_UNSUPPORTED;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(P.ctas), 1, 1);
@@ -550,12 +576,14 @@ w4a16_status launch_gemv_mma_nw(const GemvParams& P, cudaStream_t stream)
 {
     auto kern = gemv_mma_kernel<VAR, MR, NW>;
     const int smem = MgCfg<VAR, MR, NW>::smem_bytes(P.M, P.K / 32, P.g / 32);
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [&] {
-        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmemOptin);
-    });
-    if (attr_err != cudaSuccess) return W4A16_ERR_CUDA;
+    static PerDeviceInit kattr;
+    const auto set_smem = [&] {
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmemOptin);
+    };
+    if (kattr.get(set_smem) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return W4A16_ERR_CUDA;
+    }
     if (smem > kMaxSmemOptin) return W4A16_ERR_UNSUPPORTED;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(P.ctas), 1, 1);
