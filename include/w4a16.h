@@ -5,7 +5,8 @@
  *   y[M, N] = x[M, K] . (antiquant_scale (.) W)[K, N]
  *
  * with fp16 activations x, signed int4 weights W, one fp16 scale per group
- * of g consecutive K rows and per column, and an fp16 result y.  This is the
+ * of g consecutive K rows and per column, and an fp16 result y (or bf16 x,
+ * scale and y for W4A16_OP_DEQUANT_BF16 / w4a16_dequant_matmul_bf16).  This is the
  * operator of "WeightQuantBatchMatmulExperiment 算子深度解析"
  * (bjdmk.com.cn/news/4847346), section 4.2 (x float16/ND, weight int4/ND,
  * antiquant_scale float16/ND, y float16/ND, all 2-D).  Two algorithms compute it:
@@ -15,7 +16,8 @@
  *            A1..A3 from 7.49*x/A_max with two x14.98 residual steps; three
  *            exact integer matmuls Y1..Y3 against the int4 weights; combined
  *            as (Y1/7.49 + Y2/(7.49*14.98) + Y3/(7.49*14.98^2))*A_max*scale
- *            and accumulated over groups.
+ *            and accumulated over groups (2 or 4 digits instead of 3:
+ *            w4a16_msd_matmul_steps).
  *   DEQUANT  the direct dequantise-in-register W4A16 GEMM that the pages
  *            discuss as Marlin ("pwwt.cn/news/2290475", sections 1.6 and 6)
  *            and QUICK ("briefgpt.xyz/kw/cuda kernels", QUICK abstract):
