@@ -163,3 +163,15 @@ def test_moe_workspace_holds_every_intermediate(lib):
     total = lib.w4a16_moe_workspace_size(1, T, topk, K, N, g, E)
     grouped = lib.w4a16_workspace_size(1, T * topk, K, N, g, E)
     assert total >= grouped + (E + 1) * 4 + 2 * T * topk * 4 + T * topk * (K + N) * 2
+
+
+def test_binding_constants_match_the_header(lib):
+    """The op codes, device status bits and status codes the binding exposes
+    are the header's values."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    consts = {k: int(v.rstrip("u")) for k, v in re.findall(r"\b(W4A16_[A-Z0-9_]+)\s*=\s*([0-9]+u?)", text)}
+    for name in ("OP_MSD", "OP_DEQUANT", "OP_DEQUANT_BF16", "OP_MSD_2STEP", "OP_MSD_4STEP",
+                 "DEVICE_TIMEOUT", "DEVICE_BAD_EXPERT"):
+        assert getattr(lib, name) == consts["W4A16_" + name], name
+    for code, name in lib._STATUS_NAMES.items():
+        assert consts[name] == code, name

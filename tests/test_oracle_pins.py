@@ -530,3 +530,21 @@ def test_yint_planes_match_integer_gemm_and_sampled_steps_match_full():
     for S in (2, 4):
         full = oracle.msd_steps(c.x, c.wp[0], c.scale[0], 64, S)
         assert np.array_equal(oracle.msd_at_steps(c.x, c.wp[0], c.scale[0], 64, S, rows, cols), full[rows, cols])
+
+
+def test_bf16_input_encoding_is_round_to_nearest_even():
+    """The seeded bf16 inputs (inputs.to_bf16_bits) round float32 to the
+    nearest bf16, ties to even, as torch's own float32 -> bfloat16 cast does,
+    on random values and on every tie pattern of the low half-word."""
+    import torch
+    from inputs import to_bf16_bits
+    rng = np.random.default_rng(17)
+    v = np.concatenate([rng.standard_normal(20000).astype(np.float32),
+                        (rng.standard_normal(2000) * 1e-38).astype(np.float32),
+                        np.array([0.0, -0.0, 1.0, -1.0, 3.0e38, -3.0e38], np.float32)])
+    # ties: low half-word exactly 0x8000 above even and odd bf16 patterns
+    hi = rng.integers(0x0080, 0x7F00, 500).astype(np.uint32)
+    ties = ((hi << 16) | 0x8000).view(np.float32)
+    v = np.concatenate([v, ties, -ties])
+    ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(to_bf16_bits(v), ref)
