@@ -175,3 +175,25 @@ def test_binding_constants_match_the_header(lib):
         assert getattr(lib, name) == consts["W4A16_" + name], name
     for code, name in lib._STATUS_NAMES.items():
         assert consts[name] == code, name
+
+
+@pytest.mark.parametrize("lang,std", [("c", "-std=c99"), ("c++", "-std=c++11")])
+def test_header_is_plain_c_and_cxx(lang, std, tmp_path):
+    """The ABI header compiles on its own as C99 (no C++ or CUDA types leak
+    into it) and as C++11, warning-free; a C translation unit can call every
+    entry point with plain pointers."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc" if lang == "c" else "g++")
+    if cc is None:
+        pytest.skip("no host compiler")
+    src = tmp_path / ("use." + ("c" if lang == "c" else "cpp"))
+    src.write_text('#include "w4a16.h"\n'
+                   "int main(void) {\n"
+                   "    size_t ws = 0;\n"
+                   "    w4a16_status s = w4a16_workspace_size(W4A16_OP_MSD, 1, 256, 256, 128, 1, &ws);\n"
+                   "    return (int)s + (int)w4a16_packed_bytes(256, 256) * 0;\n"
+                   "}\n")
+    r = subprocess.run([cc, std, "-Wall", "-Wextra", "-Werror", "-pedantic", "-fsyntax-only",
+                        "-I", os.path.dirname(HEADER), str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
