@@ -528,6 +528,158 @@ def run_reference(args, wl, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- profiling modes (--profile)
+#
+# Not part of the benchmark line: drivers for profilers and per-variant
+# timing tables.  Every launch is the library's own.
+
+VARIANT_OPS = {"msd": 0, "dequant": 1, "bf16": 2, "msd2": 3, "msd4": 4}
+
+
+def _variant_io(torch, w4, name, variant, copies):
+    """Device inputs of one workload for one variant (bf16: the same
+    distributions encoded as bf16), weights repacked `copies` times."""
+    act = "bf16" if variant == "bf16" else "fp16"
+    c = make_workload(name, act=act)
+
+    def up(a):
+        if act == "bf16":
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+        return torch.from_numpy(a).cuda()
+    x = up(c.x)
+    wp = [[w4.repack(torch.from_numpy(p).cuda(), c.K, c.N) for p in c.wp] for _ in range(copies)]
+    sc = [up(s) for s in c.scale]
+    y = torch.empty((c.M, c.N), dtype=torch.bfloat16 if act == "bf16" else torch.float16, device="cuda")
+    op = VARIANT_OPS[variant]
+    ws = w4.alloc_workspace(op, c.M, c.K, c.N, c.g, E=c.E)
+    off = torch.from_numpy(c.offsets).cuda() if c.E > 1 else None
+
+    def call(i):
+        wpi = wp[i % copies]
+        if c.E > 1:
+            w4.w4a16_grouped_matmul(op, x, wpi, sc, off, c.E, c.M, c.K, c.N, c.g, y, ws)
+        elif variant in ("msd2", "msd4", "msd"):
+            w4.w4a16_msd_matmul_steps({"msd": 3, "msd2": 2, "msd4": 4}[variant], x, wpi[0], sc[0], c.M, c.K, c.N,
+                                      c.g, y, ws)
+        elif variant == "bf16":
+            w4.w4a16_dequant_matmul_bf16(x, wpi[0], sc[0], c.M, c.K, c.N, c.g, y, ws)
+        else:
+            w4.w4a16_dequant_matmul(x, wpi[0], sc[0], c.M, c.K, c.N, c.g, y, ws)
+    return c, call, ws
+
+
+def _graph_us(torch, fn, reps):
+    """Mean device time of `fn` over a CUDA graph of `reps` calls (fn takes
+    the call index), between two events on the capture stream."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for i in range(reps):
+                fn(i)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        g.replay()
+        e1.record(s)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1e3 / reps
+
+
+def profile_calls(args):
+    """`calls` calls of each variant in turn on the workload, rotating over
+    `calls` weight copies; checks the device status word.  For ncu."""
+    import torch
+    import weight_only_int4_a16w4_b200 as w4
+    for v in args.variants.split(","):
+        c, call, ws = _variant_io(torch, w4, args.workload, v, args.calls)
+        for i in range(args.calls):
+            call(i)
+        torch.cuda.synchronize()
+        if w4.w4a16_read_status(ws) != 0:
+            raise SystemExit("device wait timed out")
+    print("ok")
+
+
+def profile_variants(args):
+    """A markdown table of us per call for each variant on each workload (a
+    CUDA graph of consecutive calls; weights re-read from HBM: copies rotate
+    past L2 where one copy would fit)."""
+    import torch
+    import weight_only_int4_a16w4_b200 as w4
+    variants = args.variants.split(",")
+    names = args.workloads.split(",")
+    print("| workload | " + " | ".join(f"{v} us" for v in variants) + " | " +
+          " | ".join(f"{v} TFLOP/s (2MNK)" for v in variants) + " |")
+    print("|---|" + "---|" * (2 * len(variants)))
+    for name in names:
+        wl = get_workload(name)
+        b = step_bytes(wl)
+        copies = 1 if wl.E > 1 else max(2, int(np.ceil(2.2 * L2_BYTES / (b["w"] + b["scale"]))))
+        us = []
+        for v in variants:
+            c, call, ws = _variant_io(torch, w4, name, v, copies)
+            reps = 200 if wl.M * wl.N * wl.K < (1 << 36) else 10
+            reps = max(reps, copies)
+            us.append(_graph_us(torch, call, reps))
+            if w4.w4a16_read_status(ws) != 0:
+                raise SystemExit("device status set")
+        fl = step_flops(wl)
+        print(f"| {name} | " + " | ".join(f"{u:.2f}" for u in us) + " | " +
+              " | ".join(f"{fl / u / 1e6:.1f}" for u in us) + " |")
+
+
+def profile_routing(args):
+    """Routing prep of the grouped form at the grouped workload's shape: the
+    expert grouping, the row gather, the gate-weighted un-permute, and the
+    whole routed matmul next to the grouped matmul on pre-sorted rows (both
+    variants), per topk.  Router ids uniform over the experts, gate weights
+    uniform in [0, 1), seeded."""
+    import torch
+    import weight_only_int4_a16w4_b200 as w4
+    from inputs import draw_scale, draw_w, draw_x, pack_int4
+    wl = get_workload("moe_e8")
+    T, E, K, N, g = wl.M, wl.E, wl.K, wl.N, wl.g
+    rng = np.random.Generator(np.random.PCG64(20260))
+    x = torch.from_numpy(draw_x(rng, T, K)).cuda()
+    wp = [w4.repack(torch.from_numpy(pack_int4(draw_w(rng, K, N))).cuda(), K, N) for _ in range(E)]
+    sc = [torch.from_numpy(draw_scale(rng, K // g, N)).cuda() for _ in range(E)]
+    print(f"routing prep, T={T} E={E} K={K} N={N} g={g} (us per call)")
+    print("| topk | align | gather | combine | routed MSD | grouped MSD | routed dequant | grouped dequant |")
+    print("|---|---|---|---|---|---|---|---|")
+    for topk in [int(t) for t in args.topk.split(",")]:
+        rows = T * topk
+        ids = torch.from_numpy(rng.integers(0, E, (T, topk)).astype(np.int32)).cuda()
+        wts = torch.from_numpy(rng.uniform(0, 1, (T, topk)).astype(np.float32)).cuda()
+        offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+        st = torch.empty(rows, dtype=torch.int32, device="cuda")
+        inv = torch.empty(rows, dtype=torch.int32, device="cuda")
+        hdr = torch.zeros(256, dtype=torch.uint8, device="cuda")
+        xs = torch.empty((rows, K), dtype=torch.float16, device="cuda")
+        ys = torch.zeros((rows, N), dtype=torch.float16, device="cuda")
+        y = torch.empty((T, N), dtype=torch.float16, device="cuda")
+        t_align = _graph_us(torch, lambda i: w4.w4a16_moe_align(ids, T, topk, E, offsets, st, inv, hdr), 50)
+        t_gather = _graph_us(torch, lambda i: w4.w4a16_moe_gather(x, st, rows, K, xs), 20)
+        t_comb = _graph_us(torch, lambda i: w4.w4a16_moe_combine(ys, inv, wts, T, topk, N, y), 20)
+        res = []
+        for op in (w4.OP_MSD, w4.OP_DEQUANT):
+            ws = torch.zeros(w4.w4a16_moe_workspace_size(op, T, topk, K, N, g, E), dtype=torch.uint8, device="cuda")
+            gws = w4.alloc_workspace(op, rows, K, N, g, E=E)
+            res.append(_graph_us(torch, lambda i: w4.w4a16_moe_matmul(op, x, ids, wts, wp, sc, E, T, topk, K, N, g,
+                                                                      y, ws), 5))
+            res.append(_graph_us(torch, lambda i: w4.w4a16_grouped_matmul(op, xs, wp, sc, offsets, E, rows, K, N, g,
+                                                                          ys, gws), 5))
+            if w4.w4a16_read_status(ws) or w4.w4a16_read_status(gws):
+                raise SystemExit("device status set")
+        print(f"| {topk} | {t_align:.2f} | {t_gather:.2f} | {t_comb:.2f} | {res[0]:.1f} | {res[1]:.1f} | "
+              f"{res[2]:.1f} | {res[3]:.1f} |")
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -538,7 +690,24 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["calls", "variants", "routing"],
+                    help="profiler driver / timing table instead of the benchmark line")
+    ap.add_argument("--calls", type=int, default=4, help="--profile calls: calls per variant")
+    ap.add_argument("--variants", default="msd,dequant",
+                    help="--profile calls|variants: comma list of msd, dequant, bf16, msd2, msd4")
+    ap.add_argument("--workloads", default="decode_m1,decode_m16,prefill,moe_e8",
+                    help="--profile variants: comma list of workloads")
+    ap.add_argument("--topk", default="1,2", help="--profile routing: comma list of topk")
     args = ap.parse_args(argv)
+    if args.profile == "calls":
+        profile_calls(args)
+        return
+    if args.profile == "variants":
+        profile_variants(args)
+        return
+    if args.profile == "routing":
+        profile_routing(args)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world, rank, local = dist_env()

@@ -88,20 +88,30 @@ enum { W4A16_DEVICE_TIMEOUT = 1u, W4A16_DEVICE_BAD_EXPERT = 2u };
 const char* w4a16_status_string(w4a16_status s);
 
 /* Bytes of the packed (kernel-layout) weight buffer for a K x N int4 matrix:
- * ceil(N/128) * ceil(K/128) * 8192.  Equals K*N/2 when K and N are
- * multiples of 128.  Returns 0 for non-positive sizes. */
+ * ceil(N/128) * ceil(K/128) * 8192.  Equals K*N/2 -- the page's "two int4
+ * per byte" storage (bjdmk.com.cn/news/4847346, section 4.3, the int4 weight
+ * of the M=1, K=8192, N=12288 example) -- when K and N are multiples of 128;
+ * the remainder of a ragged last tile or chunk is zero padding.  Returns 0
+ * for non-positive sizes. */
 size_t w4a16_packed_bytes(int K, int N);
 
-/* Bytes of workspace a matmul call needs.
+/* Bytes of workspace a matmul call needs: the first stage of the page's
+ * two-stage call (bjdmk.com.cn/news/4847346, section 5.4: the aclnn
+ * GetWorkspaceSize query, then the execute call on a stream).
  *   op: one of the W4A16_OP_* codes; M: rows of x (for grouped calls,
  *   the total token count T); E: 1 for the dense calls, the expert count for
- *   w4a16_grouped_matmul.  The workspace holds the device status word, the
- *   split-K partial sums and arrival counters, and (MSD) the expanded
- *   activations A_int [3][M][K] int8 and A_max [K/g][M] fp32.
- * The workspace must be zero-filled before its first use; every call leaves
- * its counters at zero again, so it can be reused by later calls on the same
- * stream.  Calls that overlap in time must not share a workspace.  After a
- * call that reported a device timeout, zero it again.
+ *   w4a16_grouped_matmul.  The workspace holds the device status word (a
+ *   256-byte header) and, for MSD, the expanded activations A_int
+ *   [S][M][K] int8 and A_max [K/g][M] fp32 (the page's aUnfold workspace,
+ *   section 8.2), or on decode shapes the same digits as per-piece records.
+ *   Split-K partial sums never leave the chip (they meet in distributed
+ *   shared memory), so the workspace holds no counters.
+ * Only the status word must start at zero: zero-fill the workspace (or its
+ * first 256 bytes) before its first use.  No call writes the status word
+ * except to report a device error, so a workspace can be reused by later
+ * calls on the same stream; after a call that reported a device error, zero
+ * the status word again.  Calls that overlap in time must not share a
+ * workspace.
  * Returns W4A16_ERR_INVALID_ARG / W4A16_ERR_UNSUPPORTED on bad shapes. */
 w4a16_status w4a16_workspace_size(int op, int M, int K, int N, int group_size,
                                   int E, size_t* bytes);
@@ -286,21 +296,25 @@ w4a16_status w4a16_msd_debug_yint_steps(int steps, const void* x, const void* w_
  * host program whose memory pool owns the whole device, or a latency-critical
  * path where cudaMalloc's implicit device synchronisation is not acceptable.
  * It computes exactly what w4a16_msd_matmul computes (same kernels, same
- * arguments minus the workspace) but keeps its scratch (the expanded
- * activations, A_max, split-K partial sums and counters, status word) in one
- * array of W4A16_NOALLOC_SCRATCH_BYTES bytes that the library declares in
- * device memory; every GPU that loads the library holds that array until the
- * process exits.  It allocates nothing and calls no allocating routine.
+ * arguments minus the workspace) but keeps its scratch (the status word and
+ * the expanded activations: A_int and A_max, or the decode kernels' digit
+ * records) in one array of W4A16_NOALLOC_SCRATCH_BYTES bytes that the
+ * library declares in device memory; every GPU that loads the library holds
+ * that array until the process exits.  It allocates nothing and calls no
+ * allocating routine.
  *  - Calls whose scratch would exceed the array (see w4a16_workspace_size
  *    with W4A16_OP_MSD and E = 1) return W4A16_ERR_WORKSPACE and launch nothing.
- *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *  - The first call on a device (in a given CUDA context) looks up the
+ *    array's device address (cudaGetSymbolAddress) with that device current
+ *    and keeps it for later calls in the same context; make that first call
+ *    before any stream capture.  A call made in a context other than the one
+ *    the address was looked up in (for instance after cudaDeviceReset) looks
+ *    it up again, so it too must come before any capture.
  *  - All calls share the one array and it keeps the previous call's
- *    contents; each call zeroes the parts that must start at zero (status
- *    word, split-K counters) on `stream` before its kernels run.  Calls that
- *    may overlap on the GPU (different streams, or different host threads)
- *    race on the array: serialise them.
+ *    contents.  Only the status word must start at zero; each call zeroes it
+ *    on `stream` before its kernels run.  Calls that may overlap on the GPU
+ *    (different streams, or different host threads) race on the array:
+ *    serialise them.
  *  - A device-side wait timeout is recorded only in the array's status word,
  *    which this entry point does not report. */
 #define W4A16_NOALLOC_SCRATCH_BYTES (8u << 20)

@@ -175,6 +175,10 @@ def test_binding_constants_match_the_header(lib):
         assert getattr(lib, name) == consts["W4A16_" + name], name
     for code, name in lib._STATUS_NAMES.items():
         assert consts[name] == code, name
+    # the allocation-free entry point's array size, a macro of the form (a << b)
+    m = re.search(r"#define\s+W4A16_NOALLOC_SCRATCH_BYTES\s+\((\d+)u?\s*<<\s*(\d+)\)", text)
+    assert m, "W4A16_NOALLOC_SCRATCH_BYTES not found in the header"
+    assert lib.NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
 
 
 @pytest.mark.parametrize("lang,std", [("c", "-std=c99"), ("c++", "-std=c++11")])

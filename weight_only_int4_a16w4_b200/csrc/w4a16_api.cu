@@ -20,18 +20,6 @@
 
 using namespace w4a16;
 
-#ifdef W4A16_TRACE
-extern "C" int w4a16_trace_copy(unsigned long long* host, int n)
-{
-    if (n > 1024 * 64) n = 1024 * 64;
-    return cudaMemcpyFromSymbol(host, w4a16_trace_buf, sizeof(unsigned long long) * n) == cudaSuccess ? 0 : 1;
-}
-extern "C" int w4a16_trace_clear(const unsigned long long* zeros, int n)
-{
-    if (n > 1024 * 64) n = 1024 * 64;
-    return cudaMemcpyToSymbol(w4a16_trace_buf, zeros, sizeof(unsigned long long) * n) == cudaSuccess ? 0 : 1;
-}
-#endif
 
 namespace {
 
@@ -145,7 +133,7 @@ bool small_tile(int op, int M) { (void)op; return M <= 16; }
 // Tokens per tile.  Dequant: 256 (MMA N = 256: each MMA carries ~136 cycles
 // of tensor work, well above its issue cost -- measured 1014 vs 786 TFLOP/s
 // at M = N = K = 4096) while that still gives at least two CTAs per SM,
-// else 128.  W4A16_DEQ_TT = 128 | 256 forces one (grouped calls: T rows).
+// else 128 (grouped calls: T rows).
 // bf16 dequant: 128 (its per-group accumulators take two 128-column
 // buffers of Tensor Memory; 256 tokens would not fit beside the operand).
 int tile_tokens(int op, int M, int N)
@@ -155,12 +143,6 @@ int tile_tokens(int op, int M, int N)
     // keep two per-group accumulator buffers within Tensor Memory)
     if (is_msd_op(op)) return op_steps(op) == 4 ? 32 : 64;
     if (op == W4A16_OP_DEQUANT_BF16) return 128;
-    static int forced = -1;
-    if (forced < 0) {
-        const char* e = std::getenv("W4A16_DEQ_TT");
-        forced = (e && *e) ? std::atoi(e) : 0;
-    }
-    if (forced == 128 || forced == 256) return forced;
     return static_cast<long long>(cdiv(M, 256)) * cdiv(N, kBN) >= 2ll * sm_count() ? 256 : 128;
 }
 
@@ -251,18 +233,11 @@ int gemv_mma_smem_nw_op(int op, int NW, int M, int K, int g)
 // 32 warps): dequant at M <= 2 with N >= 8192 gains from 32 warps of one
 // quad-round each (K 4096, N 14336: 17.3 -> 16.3; K = N = 8192: 18.2 ->
 // 16.8); at N = 4096 and for MSD, 16 warps are as fast or faster (MSD
-// K 4096, N 14336: 14.7 vs 15.6); 8 warps lose everywhere.  W4A16_MG_WARPS =
-// 16 | 32 forces one.
+// K 4096, N 14336: 14.7 vs 15.6); 8 warps lose everywhere.
 int gemv_mma_warps(int op, int M, int K, int N, int g)
 {
-    static int forced = -1;
-    if (forced < 0) {
-        const char* e = std::getenv("W4A16_MG_WARPS");
-        forced = (e && *e) ? std::atoi(e) : 0;
-    }
     int nw = 16;
-    if (forced == 16 || forced == 32) nw = forced;
-    else if (!is_msd_op(op) && M <= 2 && N >= 8192) nw = 32;
+    if (!is_msd_op(op) && M <= 2 && N >= 8192) nw = 32;
     if (nw == 32 && gemv_mma_smem_nw_op(op, 32, M, K, g) > kMaxSmemOptin) nw = 16;
     return nw;
 }
@@ -280,21 +255,7 @@ int gemv_mma_smem(int op, int M, int K, int N, int g)
 //  * other g (32, 64) and M <= 4: the CUDA-core GEMV (w4a16_gemv.cuh), as the
 //    tensor tile is weak there (fp16 only: bf16 takes the decode tile);
 //  * everything else: the tensor-core decode tile.
-// W4A16_SMALL = tensor | cuda | mma forces one of them where it applies.
 enum SmallKernel { kSmallNone = 0, kSmallCuda = 1, kSmallMma = 2 };
-
-int small_override()
-{
-    static int v = -2;
-    if (v == -2) {
-        const char* e = std::getenv("W4A16_SMALL");
-        v = -1;
-        if (e && std::strcmp(e, "tensor") == 0) v = kSmallNone;
-        if (e && std::strcmp(e, "cuda") == 0) v = kSmallCuda;
-        if (e && std::strcmp(e, "mma") == 0) v = kSmallMma;
-    }
-    return v;
-}
 
 int small_kernel(int op, int M, int K, int N, int g, int E)
 {
@@ -305,10 +266,6 @@ int small_kernel(int op, int M, int K, int N, int g, int E)
     // (the CUDA-core GEMV is built for fp16 dequant and three-step MSD only)
     const bool cuda_ok = (op == W4A16_OP_DEQUANT || op == W4A16_OP_MSD) && M <= 4 &&
                          static_cast<long long>(M) * K <= kGemvMaxMK;
-    const int forced = small_override();
-    if (forced == kSmallNone) return kSmallNone;
-    if (forced == kSmallCuda) return cuda_ok ? kSmallCuda : kSmallNone;
-    if (forced == kSmallMma) return mma_ok ? kSmallMma : kSmallNone;
     if (mma_ok) return kSmallMma;
     if (cuda_ok && g % 128 != 0) return kSmallCuda;
     return kSmallNone;
@@ -356,16 +313,6 @@ w4a16_status check_shape(int M, int K, int N, int g)
 
 // ---------------------------------------------------------------- kernel launch
 
-bool use_pdl()
-{
-    static int v = -1;
-    if (v < 0) {
-        const char* e = std::getenv("W4A16_PDL");
-        v = (e && e[0] == '0') ? 0 : 1;
-    }
-    return v == 1;
-}
-
 template <int VAR, int TT, int ST, int WST, int NCONV, int NEPI, int NISS, bool SEPI, bool DBG = false>
 w4a16_status launch_gemm(const CUtensorMap& map, const GemmParams& P, dim3 grid, cudaStream_t stream)
 {
@@ -392,11 +339,9 @@ w4a16_status launch_gemm(const CUtensorMap& map, const GemmParams& P, dim3 grid,
     cfg.stream = stream;
     cudaLaunchAttribute attrs[2];
     int na = 0;
-    if (use_pdl()) {
-        attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attrs[na].val.programmaticStreamSerializationAllowed = 1;
-        ++na;
-    }
+    attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
     if (P.splits > 1) {   // the split-K CTAs of one tile form a cluster (see gemm_kernel)
         attrs[na].id = cudaLaunchAttributeClusterDimension;
         attrs[na].val.clusterDim.x = 1;
@@ -476,7 +421,7 @@ cudaError_t launch_expand_vpl(int blocks, const __half* x, int M, int K, int g, 
     attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr.val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = &attr;
-    cfg.numAttrs = use_pdl() ? 1 : 0;
+    cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, expand_kernel<VPL, S>, x, M, K, g, xq, amax);
 }
 
@@ -563,7 +508,7 @@ w4a16_status launch_gemv_mr(const GemvParams& P, cudaStream_t stream)
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = use_pdl() ? 1 : 0;
+    cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, kern, P) != cudaSuccess) {
         (void)cudaGetLastError();
         return W4A16_ERR_CUDA;
@@ -594,7 +539,7 @@ w4a16_status launch_gemv_mma_nw(const GemvParams& P, cudaStream_t stream)
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = use_pdl() ? 1 : 0;
+    cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, kern, P) != cudaSuccess) {
         (void)cudaGetLastError();
         return W4A16_ERR_CUDA;
@@ -624,7 +569,7 @@ cudaError_t launch_gemv_expand_n(const __half* x, int M, int K, int g, uint32_t*
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = use_pdl() ? 1 : 0;
+    cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, gemv_expand_kernel<NSUB, S>, x, M, K, g, rec);
 }
 
@@ -789,19 +734,50 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[W4A16_NOALLOC_S
 
 namespace {
 
-// Device address of g_noalloc_scratch on the current device, looked up once
-// per device with that device current.  nullptr on failure.
+// The driver's cuCtxGetCurrent, reached through the runtime (the library
+// does not link the driver library itself).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current_fn()
+{
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    });
+    return fn;
+}
+
+// Device address of g_noalloc_scratch on the current device, looked up with
+// that device current the first time it is needed in the current context and
+// kept per device together with the context it belongs to: a call in
+// another context (a device reset re-creates the primary context and may
+// load the module elsewhere) looks the address up again.  nullptr on failure.
 void* noalloc_scratch()
 {
     static std::mutex mu;
     static void* addr[64] = {nullptr};
+    static CUcontext owner[64] = {nullptr};
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    const CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+    if (get_ctx == nullptr) return nullptr;
+    CUcontext ctx = nullptr;   // null while the runtime has not bound a context yet
+    if (get_ctx(&ctx) != CUDA_SUCCESS) return nullptr;
     std::lock_guard<std::mutex> lock(mu);
-    if (addr[dev] == nullptr) {
+    if (ctx == nullptr || addr[dev] == nullptr || owner[dev] != ctx) {
         void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return nullptr;
+        // (binds the device's primary context if none is current yet)
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+            (void)cudaGetLastError();
+            return nullptr;
+        }
+        if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return nullptr;
         addr[dev] = p;
+        owner[dev] = ctx;
     }
     return addr[dev];
 }

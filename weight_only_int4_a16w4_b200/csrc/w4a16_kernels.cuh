@@ -46,22 +46,6 @@
 
 #include "sm100_ptx.cuh"
 
-// Optional timeline tracing (build with -DW4A16_TRACE): selected threads
-// stamp SM clock cycles at pipeline events into a per-CTA row of
-// w4a16_trace_buf, read back by the trace build's w4a16_trace_copy.
-#ifdef W4A16_TRACE
-__device__ unsigned long long w4a16_trace_buf[1024 * 64];
-#define W4A16_TRACE_AT(slot)                                                                                  \
-    do {                                                                                                      \
-        const unsigned cta_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);                \
-        if (cta_ < 1024 && (slot) < 64) w4a16_trace_buf[cta_ * 64 + (slot)] = clock64();                    \
-    } while (0)
-#else
-#define W4A16_TRACE_AT(slot) \
-    do {                     \
-    } while (0)
-#endif
-
 namespace w4a16 {
 
 constexpr int kBN = 128;                 // output columns per tile (MMA M)
@@ -502,7 +486,6 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
 
     TileCoord tc;
     if (!resolve_tile(P, TT, tc)) return;          // uniform across the CTA
-    if (threadIdx.x == 0) W4A16_TRACE_AT(1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -545,7 +528,6 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
     // The next kernel in the stream may start launching now; it waits
     // (griddep_wait) before touching anything this one writes.
     if (threadIdx.x == 0) griddep_launch_dependents();
-    if (threadIdx.x == 0) W4A16_TRACE_AT(2);
     const uint32_t tmem = *tmem_slot;
     const uint32_t tmem_a0 = tmem + C::kAccCols;               // A operand stages
     const uint64_t tmo = P.timeout_ns;
@@ -589,7 +571,6 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
                         for (int h = 0; h < srows; ++h)
                             bulk_g2s(smem_addr(ws + kWStage + h * 256), ssrc + static_cast<size_t>(sgrp0 + h) * P.N + n0,
                                      srow_bytes, fb);
-                        if (i < 8) W4A16_TRACE_AT(4 + i);
                     } else {
                         uint8_t* st = smem + s * C::kStage;
                         mbar_arrive_expect_tx(fb, C::kBBytes);
@@ -601,7 +582,6 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
                             tma_load_2d(smem_addr(st), &tmap, kc * kKC, tc.t0, fb);
                             tma_load_2d(smem_addr(st + TT * 128), &tmap, kc * kKC + 64, tc.t0, fb);
                         }
-                        if (i == 0) W4A16_TRACE_AT(3);
                     }
                 }
                 __syncwarp();
@@ -646,10 +626,8 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
                 const uint32_t ph = (i / ST) & 1;
                 const int bs = i % C::kBST;
                 const uint32_t bph = (i / C::kBST) & 1;
-                if (i == 2) W4A16_TRACE_AT(57);
                 if (!mbar_wait(smem_addr(&afull_bar[s]), ph, tmo, P.status, abort_flag)) break;
                 if (!mbar_wait(smem_addr(&bfull_bar[bs]), bph, tmo, P.status, abort_flag)) break;
-                if (i == 2) W4A16_TRACE_AT(58);
                 tc_fence_after();
                 const uint64_t bdesc = smem_desc_sw128(smem_addr(smem + bs * C::kStage));
                 const uint32_t a_base = tmem_a0 + s * C::kACols;
@@ -696,21 +674,18 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
                                 failed = true;
                                 break;
                             }
-                            if (i == 2) W4A16_TRACE_AT(59);
                             tc_fence_after();
                         }
                         const uint32_t d = tmem + ab * C::kAccStride;
                         // a group's first K step overwrites the buffer
                         if (C::kIsMsd) mma_i8_ts(d, a_base + 8 * j, bd, idesc, gpos == 0 ? 0u : 1u);
                         else mma_f16_ts(d, a_base + 8 * j, bd, idesc, gpos == 0 ? 0u : 1u);
-                        if (i == 2 && j < 4) W4A16_TRACE_AT(60 + j);
                         if (gpos == gsteps - 1) tc_commit(smem_addr(&accfull_bar[ab]));
                     } else {
                         mma_f16_ts(tmem + q * C::kAccStride, a_base + 8 * j, bd, idesc,
                                    (first_chunk && j == 0) ? 0u : 1u);
                     }
                 }
-                if (i < 8) W4A16_TRACE_AT(28 + i);
                 tc_commit(smem_addr(&sfree_bar[s]));
                 if (C::kBST != ST) tc_commit(smem_addr(&bfree_bar[bs]));
                 first_chunk = false;
@@ -735,7 +710,6 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
             const int w = i % WST;
             const uint32_t wph = (i / WST) & 1;
             if (!mbar_wait(smem_addr(&wfull_bar[w]), wph, tmo, P.status, abort_flag)) break;
-            if (cg == 0 && (warp & 3) == 0 && lane == 0 && i < 8) W4A16_TRACE_AT(12 + i);
             const uint8_t* wst = wsm + w * C::kWSlot;
             uint4 q[4];
 #pragma unroll
@@ -801,7 +775,6 @@ W4A16_ROLE_UNROLL
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_addr(&afull_bar[s]));
-            if (cg == 0 && (warp & 3) == 0 && lane == 0 && i < 8) W4A16_TRACE_AT(20 + i);
         }
     } else if (warp >= C::kEpiWarp0) {
         // ============================ epilogue ============================
@@ -850,7 +823,6 @@ W4A16_ROLE_UNROLL
                 for (int b = 0; b < C::kNBuf; ++b)
                     if (!C::kEpiRR || b % NEPI == eg) mbar_arrive(smem_addr(&accempty_bar[b]));
             griddep_wait();    // A_max comes from the expansion kernel; y is shared with earlier kernels
-            if (warp == C::kEpiWarp0 && lane == 0) W4A16_TRACE_AT(52);
 
             const int ngroups = min(kc1 * kKC, P.K) / P.g - grp0;
             const __half* sc_e = P.scale[tc.e];
@@ -894,7 +866,6 @@ W4A16_ROLE_UNROLL
                 if (C::kIsMsd) __syncwarp();
                 if (ok && !mbar_wait(smem_addr(&accfull_bar[ab]), abph, tmo, P.status, abort_flag)) ok = false;
                 if (!ok) continue;
-                if (warp == C::kEpiWarp0 && lane == 0 && j < 8) W4A16_TRACE_AT(36 + j);
                 tc_fence_after();
                 const uint32_t b_addr = t_addr + ab * C::kAccStride + tb;
                 if (C::kIsMsd) {
@@ -949,7 +920,6 @@ W4A16_ROLE_UNROLL
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_addr(&accempty_bar[ab]));
-                if (warp == C::kEpiWarp0 && lane == 0 && j < 8) W4A16_TRACE_AT(44 + j);
             }
             if (C::kEpiRR) {
                 // groups 1..NEPI-1 hand their partial sums to group 0, which
@@ -983,7 +953,6 @@ W4A16_ROLE_UNROLL
             for (int q = 0; q < nacc && ok; ++q)
                 ok = mbar_wait(smem_addr(&accfull_bar[q]), 0, tmo, P.status, abort_flag);
             if (ok) {
-                if (warp == C::kEpiWarp0 && lane == 0) W4A16_TRACE_AT(36);
                 tc_fence_after();
 #pragma unroll 1
                 for (int c = 0; c < TE / 16; ++c) {
@@ -1044,9 +1013,7 @@ W4A16_ROLE_UNROLL
     // After the barrier no CTA touches another's shared memory.
     if (C::kRedBytes > 0 && P.splits > 1) {
         __syncwarp();
-        if (warp == C::kEpiWarp0 && lane == 0) W4A16_TRACE_AT(53);
         cluster_sync_all();
-        if (warp == C::kEpiWarp0 && lane == 0) W4A16_TRACE_AT(54);
         if (warp >= C::kEpiWarp0 && P.write_y && !*abort_flag) {
             const int S = P.splits;
             const int per = (TT * kBN + S - 1) / S;
@@ -1062,12 +1029,10 @@ W4A16_ROLE_UNROLL
                 store_row<C::kBf16>(P, tc.t0 + t, nn, sum);
             }
         }
-        if (warp == C::kEpiWarp0 && lane == 0) W4A16_TRACE_AT(55);
     }
 
     tc_fence_before();
     __syncthreads();
-    if (threadIdx.x == 0) W4A16_TRACE_AT(56);
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
