@@ -337,6 +337,13 @@ def run_gpu(args, wl, rank, world, local):
     # both results come back to pinned host memory and are read.
     e2e = run_e2e(args, G, torch, w4, stream, device)
 
+    # the other M <= 16 configuration (16 tokens, N = 14336), timed per call
+    # in the same run beside the headline one
+    side = {}
+    if wl.name == "decode_m1":
+        del graph, tail
+        side["decode_m16"] = per_call_detail(w4, torch, get_workload("decode_m16"), device, stream, capture)
+
     b = step_bytes(wl)
     bytes_step = 2 * b["total"]
     flops_step = 2 * step_flops(wl)
@@ -369,6 +376,7 @@ def run_gpu(args, wl, rank, world, local):
                     "frac": round(ach_eff / peak, 4), "traffic": recorded_traffic(wl.name, dom),
                     "kernel": f"{dom} call", "peak_source": peak_kind}
 
+    detail.update(side)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6), "higher_is_better": True,
@@ -391,8 +399,45 @@ def run_gpu(args, wl, rank, world, local):
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
-        del graph, tail
+        graph = tail = None
         dist.destroy_process_group()
+
+
+def per_call_detail(w4, torch, wl, device, stream, capture):
+    """Per-call device time of each variant on another workload: a CUDA graph
+    of consecutive calls of one variant (weights rotating past L2), replayed
+    once untimed and once between two events on the launch stream."""
+    case = make_workload(wl.name)
+    G = GpuWorkload(w4, torch, wl, case, device)
+    period = max(1, G.copies // 2)
+    n_op = 2 * period * max(1, 50 // period)
+    hbm, _, _, _ = load_peaks()
+    b = step_bytes(wl)
+    out = {}
+    for op, name in ((w4.OP_MSD, "msd"), (w4.OP_DEQUANT, "dequant")):
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                G.call(op, i)
+        stream.synchronize()
+        g_op = capture(n_op, lambda s, op=op: G.call(op, s))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            g_op.replay()
+            e0.record(stream)
+            g_op.replay()
+            e1.record(stream)
+        stream.synchronize()
+        if w4.w4a16_read_status(G.ws[op], stream) != 0:
+            raise RuntimeError("device wait timed out")
+        us = e0.elapsed_time(e1) * 1e3 / n_op
+        gbs = b["total"] / (us * 1e-6) / 1e9
+        out[name] = {"us_per_call": round(us, 3), "GB/s": round(gbs, 1),
+                     "TFLOP/s": round(step_flops(wl) / (us * 1e-6) / 1e12, 2), "hbm_frac": round(gbs / hbm, 4)}
+        del g_op
+    out["config"] = f"M={wl.M} K={wl.K} N={wl.N} g={wl.g}; weights rotated over {G.copies} copies"
+    del G
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_e2e(args, G, torch, w4, stream, device):

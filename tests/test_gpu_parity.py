@@ -182,7 +182,7 @@ def test_zero_rows_is_noop(cuda_lib):
 
 
 def test_repeat_calls_are_deterministic(cuda_lib):
-    """Split-K counters reset themselves; the ordered reduction gives the
+    """The split-K partials meet in a fixed (rank) order on chip: the
     same bits on every call."""
     torch = _t()
     w4 = cuda_lib
@@ -343,8 +343,8 @@ def test_decode_tile_rows_both_variants(cuda_lib, M, K, N, g):
 
 
 def test_gemv_repeat_calls_are_deterministic(cuda_lib):
-    """The tile counters reset themselves and the partials are added in CTA
-    order, so repeated calls on one workspace give the same bits."""
+    """The warps' partial sums are added in warp order, so repeated calls on
+    one workspace give the same bits."""
     w4 = cuda_lib
     c = make_case(1, 4096, 1032, 128, seed=77)
     dev = upload(w4, c)
@@ -390,6 +390,28 @@ def _samples(rng, M, N, count):
     return rng.integers(0, M, count), rng.integers(0, N, count)
 
 
+def _tile_samples(rng, M, N, tm, tn, extra=0):
+    """One random (row, column) inside every tm x tn output tile (so a tile
+    written to the wrong place, or not at all, is caught), plus `extra`
+    uniform samples."""
+    r0 = np.arange(0, M, tm)
+    c0 = np.arange(0, N, tn)
+    rr, cc = np.meshgrid(r0, c0, indexing="ij")
+    rows = rr.ravel() + rng.integers(0, tm, rr.size)
+    cols = cc.ravel() + rng.integers(0, tn, cc.size)
+    rows, cols = np.minimum(rows, M - 1), np.minimum(cols, N - 1)
+    if extra:
+        er, ec = _samples(rng, M, N, extra)
+        rows, cols = np.concatenate([rows, er]), np.concatenate([cols, ec])
+    return rows, cols
+
+
+def assert_all_finite(y, what):
+    """The output starts as NaN: every element must have been written."""
+    bad = np.argwhere(~np.isfinite(y))
+    assert bad.size == 0, f"{what}: {len(bad)} outputs not written or not finite, first at {bad[0]}"
+
+
 def test_workload_msd_small_full(cuda_lib):
     """16 x 256 x 256, g = 64, with the forced all-zero group."""
     w4 = cuda_lib
@@ -402,54 +424,101 @@ def test_workload_msd_small_full(cuda_lib):
 
 
 def test_workload_decode_m1_full(cuda_lib):
-    """1 x 4096 x 4096, g = 128: every output checked."""
+    """1 x 4096 x 4096, g = 128: every output checked, and Y1..Y3 and A_max
+    bit-exact over every column and group -- through the kernels the
+    benchmark times (the digit-record expansion and the warp-MMA GEMV)."""
     w4 = cuda_lib
     c = make_workload(1)
     dev = upload(w4, c)
-    assert_msd_close(run_dense(w4, w4.OP_MSD, c, dev), oracle.msd(c.x, c.wp[0], c.scale[0], c.g), "msd")
-    assert_deq_close(run_dense(w4, w4.OP_DEQUANT, c, dev), oracle.dequant(c.x, c.wp[0], c.scale[0], c.g),
-                     "dequant")
-    check_yint(w4, c, dev, 0, 1, 0, 512)
+    y = run_dense(w4, w4.OP_MSD, c, dev)
+    assert_all_finite(y, "msd")
+    assert_msd_close(y, oracle.msd(c.x, c.wp[0], c.scale[0], c.g), "msd")
+    y = run_dense(w4, w4.OP_DEQUANT, c, dev)
+    assert_all_finite(y, "dequant")
+    assert_deq_close(y, oracle.dequant(c.x, c.wp[0], c.scale[0], c.g), "dequant")
+    check_yint(w4, c, dev, 0, 1, 0, c.N)
 
 
 def test_workload_decode_m16_sampled(cuda_lib):
-    """16 x 4096 x 14336, g = 128: 2048 sampled outputs plus a Y_int window."""
+    """16 x 4096 x 14336, g = 128: every output written, one sample in every
+    16 x 128 tile plus 1024 more, and Y1..Y3 bit-exact on windows at both
+    ends through the split-K decode tile the benchmark times (its cluster
+    split and both epilogue groups)."""
     w4 = cuda_lib
     c = make_workload(2)
     dev = upload(w4, c)
     rng = np.random.default_rng(2)
-    rows, cols = _samples(rng, c.M, c.N, 2048)
+    rows, cols = _tile_samples(rng, c.M, c.N, 16, 128, extra=1024)
     y = run_dense(w4, w4.OP_MSD, c, dev)
+    assert_all_finite(y, "msd")
     assert_msd_close(y[rows, cols], oracle.msd_at(c.x, c.wp[0], c.scale[0], c.g, rows, cols), "msd")
     y = run_dense(w4, w4.OP_DEQUANT, c, dev)
+    assert_all_finite(y, "dequant")
     assert_deq_close(y[rows, cols], oracle.dequant_at(c.x, c.wp[0], c.scale[0], c.g, rows, cols), "dequant")
+    check_yint(w4, c, dev, 0, 16, 0, 264)
     check_yint(w4, c, dev, 0, 16, 14336 - 136, 14336)
 
 
 def test_workload_prefill_sampled(cuda_lib):
-    """4096 x 4096 x 4096, g = 128: 2048 sampled outputs plus a Y_int window."""
+    """4096 x 4096 x 4096, g = 128: every output written, one sample in every
+    128 x 128 tile plus 1024 more, and a Y_int window."""
     w4 = cuda_lib
     c = make_workload(3)
     dev = upload(w4, c)
     rng = np.random.default_rng(3)
-    rows, cols = _samples(rng, c.M, c.N, 2048)
+    rows, cols = _tile_samples(rng, c.M, c.N, 128, 128, extra=1024)
     y = run_dense(w4, w4.OP_MSD, c, dev)
+    assert_all_finite(y, "msd")
     assert_msd_close(y[rows, cols], oracle.msd_at(c.x, c.wp[0], c.scale[0], c.g, rows, cols), "msd")
     y = run_dense(w4, w4.OP_DEQUANT, c, dev)
+    assert_all_finite(y, "dequant")
     assert_deq_close(y[rows, cols], oracle.dequant_at(c.x, c.wp[0], c.scale[0], c.g, rows, cols), "dequant")
     check_yint(w4, c, dev, 4000, 4096, 4096 - 40, 4096)
 
 
 def test_workload_moe_sampled(cuda_lib):
-    """E = 8, T = 4096, K = 4096, N = 14336: 2048 sampled outputs."""
+    """E = 8, T = 4096, K = 4096, N = 14336: every output written, one sample
+    in every 64 x 128 tile plus 1024 more."""
     w4 = cuda_lib
     c = make_workload(4)
     dev = upload(w4, c)
     rng = np.random.default_rng(4)
-    rows, cols = _samples(rng, c.M, c.N, 2048)
+    rows, cols = _tile_samples(rng, c.M, c.N, 64, 128, extra=1024)
     y = run_grouped(w4, w4.OP_MSD, c, dev)
+    assert_all_finite(y, "moe msd")
     assert_msd_close(y[rows, cols], oracle.grouped_at("msd", c.x, c.wp, c.scale, c.offsets, c.g, rows, cols),
                      "moe msd")
     y = run_grouped(w4, w4.OP_DEQUANT, c, dev)
+    assert_all_finite(y, "moe dequant")
     assert_deq_close(y[rows, cols],
                      oracle.grouped_at("dequant", c.x, c.wp, c.scale, c.offsets, c.g, rows, cols), "moe dequant")
+
+
+# ---------------------------------------------------------------- Y_int through every decode branch
+
+# (M, K, N, g, kernel the product call dispatches to for MSD)
+YINT_BRANCHES = [
+    (1, 4096, 4096, 128, "warp-MMA GEMV, one token"),
+    (2, 2048, 1032, 256, "warp-MMA GEMV, two tokens, 256-deep groups cut between warps, ragged column blocks"),
+    (1, 14336, 512, 128, "warp-MMA GEMV, several quads per warp"),
+    (1, 1024, 4096, 64, "CUDA-core dp4a GEMV, g = 64"),
+    (3, 2048, 520, 32, "CUDA-core dp4a GEMV, g = 32, three tokens"),
+    (4, 4096, 4096, 128, "split-K decode tile (cluster of K ranges), four tokens"),
+    (16, 4096, 2048, 128, "split-K decode tile, 16 tokens"),
+    (9, 1024, 264, 64, "decode tile, g = 64, K split over a cluster of 8, ragged N"),
+    (40, 512, 392, 128, "64-token tile, ragged tokens and columns"),
+]
+
+
+@pytest.mark.parametrize("M,K,N,g,branch", YINT_BRANCHES, ids=[b[4] for b in YINT_BRANCHES])
+def test_yint_bit_exact_on_every_branch(cuda_lib, M, K, N, g, branch):
+    """Equation 9's per-group int32 Y1..Y3 and A_max, bit-exact against the
+    oracle, read back from the kernels the product MSD call runs for this
+    shape (the debug window runs the same kernels and launch shapes), over
+    every row, group and column."""
+    w4 = cuda_lib
+    c = make_case(M, K, N, g, seed=4100 + M + N)
+    dev = upload(w4, c)
+    check_yint(w4, c, dev, 0, M, 0, N)
+    # and the product call on the same inputs is within the MSD bar
+    assert_msd_close(run_dense(w4, w4.OP_MSD, c, dev), oracle.msd(c.x, c.wp[0], c.scale[0], g), branch)

@@ -375,9 +375,10 @@ w4a16_status launch_gemm(const CUtensorMap& map, const GemmParams& P, dim3 grid,
 w4a16_status launch_for(int op, int TT, const CUtensorMap& map, const GemmParams& P, dim3 grid, cudaStream_t s)
 {
     if (op == W4A16_OP_MSD) {
-        // the Y_int debug window is a separate instance, off the hot kernels
+        // the Y_int debug window: the product instance's template parameters
+        // with the window writes switched on
         if (P.dbg_yint != nullptr) {
-            if (TT == 16) return launch_gemm<kMsd, 16, 8, 12, 2, 1, 4, false, true>(map, P, grid, s);
+            if (TT == 16) return launch_gemm<kMsd, 16, 8, 12, 2, 2, 4, false, true>(map, P, grid, s);
             return launch_gemm<kMsd, 64, 4, 4, 2, 2, 1, false, true>(map, P, grid, s);
         }
         if (TT == 16) return launch_gemm<kMsd, 16, 8, 12, 2, 2, 4, false>(map, P, grid, s);
@@ -385,7 +386,7 @@ w4a16_status launch_for(int op, int TT, const CUtensorMap& map, const GemmParams
     }
     if (op == W4A16_OP_MSD_2STEP) {
         if (P.dbg_yint != nullptr) {
-            if (TT == 16) return launch_gemm<kMsd2, 16, 8, 12, 2, 1, 4, false, true>(map, P, grid, s);
+            if (TT == 16) return launch_gemm<kMsd2, 16, 8, 12, 2, 2, 4, false, true>(map, P, grid, s);
             return launch_gemm<kMsd2, 64, 4, 4, 2, 2, 1, false, true>(map, P, grid, s);
         }
         if (TT == 16) return launch_gemm<kMsd2, 16, 8, 12, 2, 2, 4, false>(map, P, grid, s);
@@ -394,7 +395,7 @@ w4a16_status launch_for(int op, int TT, const CUtensorMap& map, const GemmParams
     if (op == W4A16_OP_MSD_4STEP) {
         // 4 x 16-row activation stages: 8 weight stages keep shared memory in bounds
         if (P.dbg_yint != nullptr) {
-            if (TT == 16) return launch_gemm<kMsd4, 16, 8, 8, 2, 1, 4, false, true>(map, P, grid, s);
+            if (TT == 16) return launch_gemm<kMsd4, 16, 8, 8, 2, 2, 4, false, true>(map, P, grid, s);
             return launch_gemm<kMsd4, 32, 4, 4, 2, 2, 1, false, true>(map, P, grid, s);
         }
         if (TT == 16) return launch_gemm<kMsd4, 16, 8, 8, 2, 2, 4, false>(map, P, grid, s);
@@ -484,11 +485,11 @@ void base_params(GemmParams& P, int op, int M, int K, int N, int g, const Shape&
     P.write_y = 1;
 }
 
-template <int VAR, int MR>
+template <int VAR, int MR, bool DBG = false>
 w4a16_status launch_gemv_mr(const GemvParams& P, cudaStream_t stream)
 {
     using C = GemvCfg<VAR, MR>;
-    auto kern = gemv_kernel<VAR, MR>;
+    auto kern = gemv_kernel<VAR, MR, DBG>;
     const int smem = C::smem_bytes(P.M, P.K);
     static PerDeviceInit kattr;
     const auto set_smem = [&] {
@@ -516,10 +517,10 @@ w4a16_status launch_gemv_mr(const GemvParams& P, cudaStream_t stream)
     return W4A16_OK;
 }
 
-template <int VAR, int MR, int NW>
+template <int VAR, int MR, int NW, bool DBG = false>
 w4a16_status launch_gemv_mma_nw(const GemvParams& P, cudaStream_t stream)
 {
-    auto kern = gemv_mma_kernel<VAR, MR, NW>;
+    auto kern = gemv_mma_kernel<VAR, MR, NW, DBG>;
     const int smem = MgCfg<VAR, MR, NW>::smem_bytes(P.M, P.K / 32, P.g / 32);
     static PerDeviceInit kattr;
     const auto set_smem = [&] {
@@ -547,13 +548,13 @@ w4a16_status launch_gemv_mma_nw(const GemvParams& P, cudaStream_t stream)
     return W4A16_OK;
 }
 
-template <int VAR, int MR>
+template <int VAR, int MR, bool DBG = false>
 w4a16_status launch_gemv_mma_mr(const GemvParams& P, cudaStream_t stream)
 {
     const int op = VAR == kMsd ? W4A16_OP_MSD : VAR == kMsd2 ? W4A16_OP_MSD_2STEP
                  : VAR == kMsd4 ? W4A16_OP_MSD_4STEP : W4A16_OP_DEQUANT;
-    if (gemv_mma_warps(op, P.M, P.K, P.N, P.g) == 32) return launch_gemv_mma_nw<VAR, MR, 32>(P, stream);
-    return launch_gemv_mma_nw<VAR, MR, 16>(P, stream);
+    if (gemv_mma_warps(op, P.M, P.K, P.N, P.g) == 32) return launch_gemv_mma_nw<VAR, MR, 32, DBG>(P, stream);
+    return launch_gemv_mma_nw<VAR, MR, 16, DBG>(P, stream);
 }
 
 template <int NSUB, int S>
@@ -585,25 +586,41 @@ cudaError_t launch_gemv_expand_s(const __half* x, int M, int K, int g, uint32_t*
     }
 }
 
-// the warp-MMA GEMV of an MSD variant, MR chosen by M
-template <int VAR>
-w4a16_status launch_gemv_mma_msd(const GemvParams& P, int op, cudaStream_t stream)
+// the warp-MMA GEMV of an MSD variant, MR chosen by M; DBG: the Y_int
+// window instance
+template <int VAR, bool DBG>
+w4a16_status launch_gemv_mma_msd_dbg(const GemvParams& P, int op, cudaStream_t stream)
 {
     switch (gemv_mma_rows(op, P.M)) {
-        case 1: return launch_gemv_mma_mr<VAR, 1>(P, stream);
-        case 2: return launch_gemv_mma_mr<VAR, 2>(P, stream);
+        case 1: return launch_gemv_mma_mr<VAR, 1, DBG>(P, stream);
+        case 2: return launch_gemv_mma_mr<VAR, 2, DBG>(P, stream);
         default:
-            if constexpr (4 * msd_steps(VAR) <= 8) return launch_gemv_mma_mr<VAR, 4>(P, stream);
+            if constexpr (4 * msd_steps(VAR) <= 8) return launch_gemv_mma_mr<VAR, 4, DBG>(P, stream);
             return W4A16_ERR_UNSUPPORTED;
     }
 }
 
+template <int VAR>
+w4a16_status launch_gemv_mma_msd(const GemvParams& P, int op, cudaStream_t stream)
+{
+    return P.dbg_yint != nullptr ? launch_gemv_mma_msd_dbg<VAR, true>(P, op, stream)
+                                 : launch_gemv_mma_msd_dbg<VAR, false>(P, op, stream);
+}
+
 w4a16_status launch_gemv(int op, bool mma, const void* x, const void* w_packed, const void* scale, int M, int K, int N,
-                         int g, void* y, void* ws, const Shape& s, const WsLayout& L, cudaStream_t stream)
+                         int g, void* y, void* ws, const Shape& s, const WsLayout& L, cudaStream_t stream,
+                         int32_t* dbg_yint = nullptr, float* dbg_amax = nullptr, int m0 = 0, int m1 = 0, int n0 = 0,
+                         int n1 = 0)
 {
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     GemvParams P;
     std::memset(&P, 0, sizeof(P));
+    P.dbg_yint = dbg_yint;
+    P.dbg_amax = dbg_amax;
+    P.dbg_m0 = m0;
+    P.dbg_m1 = m1;
+    P.dbg_n0 = n0;
+    P.dbg_n1 = n1;
     P.x = static_cast<const __half*>(x);
     P.w = static_cast<const uint8_t*>(w_packed);
     P.scale = static_cast<const __half*>(scale);
@@ -639,6 +656,11 @@ w4a16_status launch_gemv(int op, bool mma, const void* x, const void* w_packed, 
                 case 4: return launch_gemv_mma_msd<kMsd4>(P, op, stream);
                 default: return launch_gemv_mma_msd<kMsd>(P, op, stream);
             }
+        }
+        if (P.dbg_yint != nullptr) {
+            if (M == 1) return launch_gemv_mr<kMsd, 1, true>(P, stream);
+            if (M == 2) return launch_gemv_mr<kMsd, 2, true>(P, stream);
+            return launch_gemv_mr<kMsd, 4, true>(P, stream);
         }
         if (M == 1) return launch_gemv_mr<kMsd, 1>(P, stream);
         if (M == 2) return launch_gemv_mr<kMsd, 2>(P, stream);
@@ -680,11 +702,9 @@ w4a16_status dense_matmul(int op, const void* x, const void* w_packed, const voi
     if (!aligned16(x) || !aligned16(w_packed) || (scale && !aligned16(scale)) || (y && !aligned16(y)) ||
         !aligned16(ws))
         return W4A16_ERR_INVALID_ARG;
-    Shape s = dense_shape(op, M, K, N, g);
-    const WsLayout full = ws_layout(op, s, M, K, N, g);
-    if (debug) s.splits = 1;
+    const Shape s = dense_shape(op, M, K, N, g);
     const WsLayout L = ws_layout(op, s, M, K, N, g);
-    if (ws_bytes < full.total) return W4A16_ERR_WORKSPACE;
+    if (ws_bytes < L.total) return W4A16_ERR_WORKSPACE;
 
     GemmParams P;
     base_params(P, op, M, K, N, g, s, ws);
@@ -701,9 +721,18 @@ w4a16_status dense_matmul(int op, const void* x, const void* w_packed, const voi
         P.dbg_n0 = n0;
         P.dbg_n1 = n1;
     }
-    if (!debug) {
+    // the debug window runs the very kernels (and launch shapes) of the
+    // product call, in instances that write Y_int instead of y; the GEMV adds
+    // parts of a group into it, so it starts at zero
+    if (debug) {
+        const size_t wbytes = static_cast<size_t>(op_steps(op)) * (m1 - m0) * (K / g) * (n1 - n0) * sizeof(int32_t);
+        if (cudaMemsetAsync(dbg_yint, 0, wbytes, stream) != cudaSuccess) return W4A16_ERR_CUDA;
+    }
+    {
         const int sk = small_kernel(op, M, K, N, g, 1);
-        if (sk != kSmallNone) return launch_gemv(op, sk == kSmallMma, x, w_packed, scale, M, K, N, g, y, ws, s, L, stream);
+        if (sk != kSmallNone)
+            return launch_gemv(op, sk == kSmallMma, x, w_packed, scale, M, K, N, g, y, ws, s, L, stream, dbg_yint,
+                               dbg_amax, m0, m1, n0, n1);
     }
     CUtensorMap map;
     if (is_msd_op(op)) {

@@ -67,7 +67,25 @@ struct GemvParams {
     int npieces;              // K / 32
     int nblk;                 // ceil(N / 32)
     int ctas;                 // P
+    // MSD Y_int debug window (DBG instances only): int32 [S][m1-m0][G][n1-n0]
+    // and A_max fp32 [m1-m0][G]; no scale is read and no y is written
+    int32_t* dbg_yint;
+    float* dbg_amax;
+    int dbg_m0, dbg_m1, dbg_n0, dbg_n1;
 };
+
+// One MSD Y_i (plane p of token m, group grp, column n) into the debug
+// window, if it lies there.  ATOMIC: a group's sum arrives in parts (from
+// several warps) and is added up exactly in int32 (the window starts at 0).
+template <bool ATOMIC>
+__device__ __forceinline__ void dbg_put_yint(const GemvParams& P, int p, int m, int grp, int n, int y)
+{
+    if (m < P.dbg_m0 || m >= P.dbg_m1 || n < P.dbg_n0 || n >= P.dbg_n1) return;
+    const int wm = P.dbg_m1 - P.dbg_m0, wn = P.dbg_n1 - P.dbg_n0;
+    int32_t* dst = P.dbg_yint + ((static_cast<size_t>(p) * wm + (m - P.dbg_m0)) * P.G + grp) * wn + (n - P.dbg_n0);
+    if (ATOMIC) atomicAdd(dst, y);
+    else *dst = y;
+}
 
 template <int VAR, int MR>
 struct GemvCfg {
@@ -246,7 +264,7 @@ __global__ void __launch_bounds__(256) gemv_expand_kernel(const __half* __restri
 
 // ------------------------------------------------------------------ the GEMV
 
-template <int VAR, int MR>
+template <int VAR, int MR, bool DBG = false>
 __global__ void __launch_bounds__(kGemvThreads, 2) gemv_kernel(const __grid_constant__ GemvParams P)
 {
     using C = GemvCfg<VAR, MR>;
@@ -292,7 +310,7 @@ __global__ void __launch_bounds__(kGemvThreads, 2) gemv_kernel(const __grid_cons
             if (p < pw1) {
                 buf[j] = ldg_stream(wt + static_cast<size_t>(p >> 2) * kWStage + (p & 3) * 2048);
                 if (++pos == ppg) {
-                    if (n < P.N) h = __half_as_ushort(P.scale[static_cast<size_t>(grp) * P.N + n]);
+                    if (n < P.N && !DBG) h = __half_as_ushort(P.scale[static_cast<size_t>(grp) * P.N + n]);
                     ++grp;
                     pos = 0;
                 }
@@ -356,6 +374,19 @@ __global__ void __launch_bounds__(kGemvThreads, 2) gemv_kernel(const __grid_cons
                 if (group_end) {
                     const float scl =
                         __half2float(__ushort_as_half(static_cast<unsigned short>(sc[j >> 1] >> (16 * (j & 1)))));
+                    if constexpr (DBG) {
+                        // warps take whole groups: yacc is the group's Y_i
+                        const int n = (b0 + i / rpb) * 32 + lane;
+#pragma unroll
+                        for (int m = 0; m < MR; ++m) {
+                            if (m >= M) break;
+#pragma unroll
+                            for (int pl = 0; pl < 3; ++pl) dbg_put_yint<false>(P, pl, m, grp, n, yacc[m][pl]);
+                            if (n == P.dbg_n0 && m >= P.dbg_m0 && m < P.dbg_m1)
+                                P.dbg_amax[static_cast<size_t>(m - P.dbg_m0) * P.G + grp] =
+                                    __uint_as_float(rec_s[(static_cast<size_t>(p) * M + m) * kGemvRecWords + 27]);
+                        }
+                    }
 #pragma unroll
                     for (int m = 0; m < MR; ++m) {
                         if (m >= M) break;
@@ -413,7 +444,7 @@ __global__ void __launch_bounds__(kGemvThreads, 2) gemv_kernel(const __grid_cons
             if (tid < 32 * MR) {
                 const int m = tid >> 5, l = tid & 31;
                 const int n = (b0 + i / rpb) * 32 + l;
-                if (m < M && n < P.N) {
+                if (m < M && n < P.N && !DBG) {
                     float s = 0.f;
 #pragma unroll
                     for (int w = 0; w < kGemvWarps; ++w) s += red[(w * MR + m) * 32 + l];

@@ -183,7 +183,7 @@ __device__ __forceinline__ void unpack_exact_f16(uint32_t q, uint32_t (&p)[4])
     p[3] = *reinterpret_cast<const uint32_t*>(&w3);
 }
 
-template <int VAR, int MR, int NW>
+template <int VAR, int MR, int NW, bool DBG = false>
 __global__ void __launch_bounds__(NW * 32, NW >= 32 ? 1 : 2) gemv_mma_kernel(const __grid_constant__ GemvParams P)
 {
     using C = MgCfg<VAR, MR, NW>;
@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(NW * 32, NW >= 32 ? 1 : 2) gemv_mma_kernel(con
                     cp_async16(smem_addr(ring + (slot * 4 + j) * 512 + ((lane ^ (2 * j)) * 16)), src + j * 2048);
             }
             const int b = b0 + bg * kMgCB + lane;
-            if (lane < kMgCB && b < b1)
+            if (lane < kMgCB && b < b1 && !DBG)
                 cp_async16(smem_addr(sring + (slot * kMgCB + lane) * 16),
                            P.scale + static_cast<size_t>(grp) * P.N + b * 8);
         }
@@ -309,6 +309,25 @@ __global__ void __launch_bounds__(NW * 32, NW >= 32 ? 1 : 2) gemv_mma_kernel(con
                     }
                 }
                 if (closes) {
+                    if constexpr (DBG) {
+                        // the warp's part of the group's Y_i (a group may be cut
+                        // between two warps: the window adds the parts exactly)
+                        if (row_ok) {
+                            const int grp = (4 * q) / ppg;
+#pragma unroll
+                            for (int k = 0; k < kMgCB; ++k) {
+                                if (k >= nbk) break;
+                                const int n = (bb + k) * 8 + 2 * tl;
+                                dbg_put_yint<true>(P, row_plane, row_m, grp, n, d[k][0] + corr);
+                                dbg_put_yint<true>(P, row_plane, row_m, grp, n + 1, d[k][1] + corr);
+                            }
+                            const int nb0 = P.dbg_n0 / 8;
+                            if (row_plane == 0 && tl == 0 && nb0 >= bb && nb0 < bb + nbk && row_m >= P.dbg_m0 &&
+                                row_m < P.dbg_m1)
+                                P.dbg_amax[static_cast<size_t>(row_m - P.dbg_m0) * P.G + grp] =
+                                    __uint_as_float(r[9 * C::kS]);
+                        }
+                    }
                     // word 9S of a record is the A_max of its group
                     const float alpha = row_ok ? row_c * __uint_as_float(r[9 * C::kS]) : 0.f;   // rows past S M: unused
 #pragma unroll
@@ -389,7 +408,7 @@ __global__ void __launch_bounds__(NW * 32, NW >= 32 ? 1 : 2) gemv_mma_kernel(con
                         s += rw[m * 8];
                     }
                 }
-                store_elem<C::kBf16>(P.y + static_cast<size_t>(m) * P.N + (bb + k) * 8 + col, s);
+                if (!DBG) store_elem<C::kBf16>(P.y + static_cast<size_t>(m) * P.N + (bb + k) * 8 + col, s);
             }
             if (bg + 1 < nbg) __syncthreads();
 #pragma unroll

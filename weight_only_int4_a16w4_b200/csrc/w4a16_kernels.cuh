@@ -971,16 +971,21 @@ W4A16_ROLE_UNROLL
 #pragma unroll
                         for (int k = 0; k < 16; ++k) v[k] += __uint_as_float(u[k]);
                     }
+                    // the routed/dense choice is made once per chunk of 16
+                    // tokens, outside the unrolled stores: the dense path
+                    // runs plain stores only
                     if (P.write_y && n_ok) {
+                        if (P.row_dst == nullptr) {
+                            __half* yp = P.y + static_cast<size_t>(tc.t0 + tb + 16 * c) * P.N + n;
+                            const int kmax = nt - (tb + 16 * c);
 #pragma unroll
-                        for (int k = 0; k < 16; ++k)
-                            if (tb + 16 * c + k < nt) {
-                                if (P.row_dst == nullptr)
-                                    store_elem<C::kBf16>(P.y + static_cast<size_t>(tc.t0 + tb + 16 * c + k) * P.N + n,
-                                                         v[k]);
-                                else
-                                    store_mapped(tb + 16 * c + k, v[k]);
-                            }
+                            for (int k = 0; k < 16; ++k)
+                                if (k < kmax) store_elem<C::kBf16>(yp + static_cast<size_t>(k) * P.N, v[k]);
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < 16; ++k)
+                                if (tb + 16 * c + k < nt) store_mapped(tb + 16 * c + k, v[k]);
+                        }
                     }
                 }
                 tc_fence_before();
