@@ -184,6 +184,29 @@ struct GemmCfg {
     static_assert(!kEpiRR || (kGroupAcc && kNBuf % NEPI == 0), "round-robin epilogue needs per-group buffers");
 };
 
+// two fp32 lanes at once (sm_100 packed fp32): a * b + c and a * b, each lane
+// rounded as the scalar instruction would
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
 // ------------------------------------------------------------------ helpers
 
 __device__ __forceinline__ uint32_t pack_half2_bits(__half2 h)
@@ -880,14 +903,18 @@ W4A16_ROLE_UNROLL
                         const float am[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
                         tmem_ld_wait();
 #pragma unroll
-                        for (int qq = 0; qq < 8; ++qq) {
-                            // exact Y_i as floats (|Y| < 2^22 < 2^24), then equation 10
-                            // and equation 11's running sum
-                            float v = __int2float_rn(static_cast<int>(yv[0][qq]));
+                        for (int qq = 0; qq < 8; qq += 2) {
+                            float2 v = make_float2(__int2float_rn(static_cast<int>(yv[0][qq])),
+                                                   __int2float_rn(static_cast<int>(yv[0][qq + 1])));
 #pragma unroll
                             for (int p = 1; p < C::kVals; ++p)
-                                v = fmaf(__int2float_rn(static_cast<int>(yv[p][qq])), msd_plane_r(p), v);
-                            acc[8 * c + qq] = fmaf(v, am[qq] * scc, acc[8 * c + qq]);
+                                v = ffma2(make_float2(__int2float_rn(static_cast<int>(yv[p][qq])),
+                                                      __int2float_rn(static_cast<int>(yv[p][qq + 1]))),
+                                          make_float2(msd_plane_r(p), msd_plane_r(p)), v);
+                            const float2 f = fmul2(make_float2(am[qq], am[qq + 1]), make_float2(scc, scc));
+                            const float2 a = ffma2(v, f, make_float2(acc[8 * c + qq], acc[8 * c + qq + 1]));
+                            acc[8 * c + qq] = a.x;
+                            acc[8 * c + qq + 1] = a.y;
                         }
                         if (DBG && n_ok && n >= P.dbg_n0 && n < P.dbg_n1) {
                             const int wn = P.dbg_n1 - P.dbg_n0, wm = P.dbg_m1 - P.dbg_m0;
