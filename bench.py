@@ -281,14 +281,38 @@ def run_gpu(args, wl, rank, world, local):
                     body(s)
         return g
 
-    graph = capture(per_graph, G.step) if nrep else None
-    tail = capture(rem, G.step) if rem else None
-    # untimed replay to warm the graph
+    # The timed region's start and stop events are nodes of the captured
+    # graphs themselves (the first node of the first graph, the last node of
+    # the last), so the window holds exactly the K steps as the device runs
+    # them, not the host's submission of the graph; the K steps run as: the
+    # first graph, nrep - 1 more full graphs, then the remainder.
+    t0 = torch.cuda.Event(enable_timing=True, external=True)
+    t1 = torch.cuda.Event(enable_timing=True, external=True)
+
+    def capture_timed(n, start, stop):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                if start:
+                    t0.record(stream)
+                for s in range(n):
+                    G.step(s)
+                if stop:
+                    t1.record(stream)
+        return g
+
+    if nrep == 0:
+        timed = [capture_timed(rem, True, True)]
+        graph = tail = None
+    else:
+        first = capture_timed(per_graph, True, rem == 0 and nrep == 1)
+        graph = capture(per_graph, G.step) if nrep > 1 else None
+        tail = capture_timed(rem, False, True) if (rem or nrep > 1) else None
+        timed = [first] + [graph] * (nrep - 1) + ([tail] if tail is not None else [])
+    # untimed replay to warm the graphs
     with torch.cuda.stream(stream):
-        if graph is not None:
-            graph.replay()
-        if tail is not None:
-            tail.replay()
+        for gr in {id(gr): gr for gr in timed}.values():
+            gr.replay()
     stream.synchronize()
 
     sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
@@ -296,14 +320,9 @@ def run_gpu(args, wl, rank, world, local):
     time.sleep(0.3)
     barrier(device)
     torch.cuda.synchronize()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
-        t0.record(stream)
-        for _ in range(nrep):
-            graph.replay()
-        if tail is not None:
-            tail.replay()
-        t1.record(stream)
+        for gr in timed:
+            gr.replay()
     stream.synchronize()
     barrier(device)
     torch.cuda.synchronize()
@@ -341,7 +360,7 @@ def run_gpu(args, wl, rank, world, local):
     # in the same run beside the headline one
     side = {}
     if wl.name == "decode_m1":
-        del graph, tail
+        del graph, tail, timed
         side["decode_m16"] = per_call_detail(w4, torch, get_workload("decode_m16"), device, stream, capture)
 
     b = step_bytes(wl)
@@ -385,8 +404,9 @@ def run_gpu(args, wl, rank, world, local):
         "config": {"workload": f"{wl.name}: M={wl.M} K={wl.K} N={wl.N} g={wl.g}" + (f" E={wl.E}" if wl.E > 1 else "")
                    + "; one step = MSD matmul + dequant matmul",
                    "l2": f"weights rotated over {G.copies} copies (> L2) between calls",
-                   "timing": f"CUDA graph of {per_graph} steps replayed; events on the launch stream; per-call times from "
-                             f"graphs of {n_op} calls of one variant",
+                   "timing": f"{args.steps} steps as CUDA graphs of up to {per_graph} steps, the start and stop "
+                             f"events being nodes of the first and last graph; per-call times from graphs of {n_op} "
+                             f"calls of one variant",
                    "parallelism": f"{world} independent replica(s), one per GPU" if world > 1 else "single GPU",
                    "tflops_per_s": round(flops_step * args.steps * world / (ms * 1e-3) / 1e12, 3)},
         "roofline": roof, "detail": detail, "e2e": e2e,
@@ -399,7 +419,7 @@ def run_gpu(args, wl, rank, world, local):
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
-        graph = tail = None
+        graph = tail = timed = None
         dist.destroy_process_group()
 
 
