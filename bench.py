@@ -356,12 +356,17 @@ def run_gpu(args, wl, rank, world, local):
     # both results come back to pinned host memory and are read.
     e2e = run_e2e(args, G, torch, w4, stream, device)
 
-    # the other M <= 16 configuration (16 tokens, N = 14336), timed per call
-    # in the same run beside the headline one
+    # the other configurations, timed per call in the same run beside the
+    # headline one: decode_m16 (the other M <= 16 case) against the copy
+    # bandwidth, prefill and moe_e8 against the tensor-pipe peaks
     side = {}
+    main_copies, main_grouped = G.copies, G.grouped
     if wl.name == "decode_m1":
         del graph, tail, timed
-        side["decode_m16"] = per_call_detail(w4, torch, get_workload("decode_m16"), device, stream, capture)
+        del G
+        torch.cuda.empty_cache()
+        for other in ("decode_m16", "prefill", "moe_e8"):
+            side[other] = per_call_detail(w4, torch, get_workload(other), device, stream, capture)
 
     b = step_bytes(wl)
     bytes_step = 2 * b["total"]
@@ -403,14 +408,14 @@ def run_gpu(args, wl, rank, world, local):
         "data": "synthetic (seeded; x ~ N(0,1) fp16 with 0.1% x20 outliers, w ~ U{-8..7}, scale ~ U[0.005,0.02])",
         "config": {"workload": f"{wl.name}: M={wl.M} K={wl.K} N={wl.N} g={wl.g}" + (f" E={wl.E}" if wl.E > 1 else "")
                    + "; one step = MSD matmul + dequant matmul",
-                   "l2": f"weights rotated over {G.copies} copies (> L2) between calls",
+                   "l2": f"weights rotated over {main_copies} copies (> L2) between calls",
                    "timing": f"{args.steps} steps as CUDA graphs of up to {per_graph} steps, the start and stop "
                              f"events being nodes of the first and last graph; per-call times from graphs of {n_op} "
                              f"calls of one variant",
                    "parallelism": f"{world} independent replica(s), one per GPU" if world > 1 else "single GPU",
                    "tflops_per_s": round(flops_step * args.steps * world / (ms * 1e-3) / 1e12, 3)},
         "roofline": roof, "detail": detail, "e2e": e2e,
-        "gpu_launches": launches_per_step(G.grouped) * args.steps,
+        "gpu_launches": launches_per_step(main_grouped) * args.steps,
         "clocks": clocks, "kernel_sha": kernel_sha(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -434,6 +439,7 @@ def per_call_detail(w4, torch, wl, device, stream, capture):
     hbm, _, _, _ = load_peaks()
     b = step_bytes(wl)
     out = {}
+    _, bf16_peak, _, _ = load_peaks()
     for op, name in ((w4.OP_MSD, "msd"), (w4.OP_DEQUANT, "dequant")):
         with torch.cuda.stream(stream):
             for i in range(3):
@@ -451,8 +457,14 @@ def per_call_detail(w4, torch, wl, device, stream, capture):
             raise RuntimeError("device wait timed out")
         us = e0.elapsed_time(e1) * 1e3 / n_op
         gbs = b["total"] / (us * 1e-6) / 1e9
-        out[name] = {"us_per_call": round(us, 3), "GB/s": round(gbs, 1),
-                     "TFLOP/s": round(step_flops(wl) / (us * 1e-6) / 1e12, 2), "hbm_frac": round(gbs / hbm, 4)}
+        tfl = step_flops(wl) / (us * 1e-6) / 1e12
+        out[name] = {"us_per_call": round(us, 3), "GB/s": round(gbs, 1), "TFLOP/s": round(tfl, 2),
+                     "hbm_frac": round(gbs / hbm, 4)}
+        if wl.M > 16:
+            # MSD: its 6 M N K int8 ops against the int8 peak (2 x the bf16
+            # one); dequant: 2 M N K fp16 flops against the bf16 peak
+            out[name]["tensor_frac"] = round(tfl * (3.0 if name == "msd" else 1.0) /
+                                             (bf16_peak * (2.0 if name == "msd" else 1.0)), 4)
         del g_op
     out["config"] = f"M={wl.M} K={wl.K} N={wl.N} g={wl.g}; weights rotated over {G.copies} copies"
     del G
