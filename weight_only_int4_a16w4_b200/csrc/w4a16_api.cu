@@ -441,6 +441,42 @@ cudaError_t launch_expand_s(int blocks, const __half* xh, int M, int K, int g, i
     }
 }
 
+template <int S, int STEPS>
+cudaError_t launch_expand8(const __half* x, int M, int K, int g, int8_t* xq, float* amax, cudaStream_t s)
+{
+    // warp tasks of STEPS * 256 values; at most 8 CTAs of 8 warps per SM,
+    // the warps loop over the rest
+    const long long tasks = (static_cast<long long>(M) * K / 8 + 32 * STEPS - 1) / (32 * STEPS);
+    const int blocks = static_cast<int>(std::min<long long>((tasks + 7) / 8, 8ll * sm_count()));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(blocks, 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    switch (g / 8) {
+        case 4: return cudaLaunchKernelEx(&cfg, expand8_kernel<4, S, STEPS>, x, M, K, g, xq, amax);
+        case 8: return cudaLaunchKernelEx(&cfg, expand8_kernel<8, S, STEPS>, x, M, K, g, xq, amax);
+        case 16: return cudaLaunchKernelEx(&cfg, expand8_kernel<16, S, STEPS>, x, M, K, g, xq, amax);
+        case 32: return cudaLaunchKernelEx(&cfg, expand8_kernel<32, S, STEPS>, x, M, K, g, xq, amax);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+// Four 256-value blocks per warp task once that still gives every SM 64
+// warps' worth of tasks (large M: more loads in flight per warp); one block
+// per task below that, where the warps' count matters more.
+template <int S>
+cudaError_t launch_expand8_s(const __half* x, int M, int K, int g, int8_t* xq, float* amax, cudaStream_t s)
+{
+    const long long tasks4 = (static_cast<long long>(M) * K / 8 + 127) / 128;
+    if (tasks4 >= 64ll * sm_count()) return launch_expand8<S, 4>(x, M, K, g, xq, amax, s);
+    return launch_expand8<S, 1>(x, M, K, g, xq, amax, s);
+}
+
 w4a16_status launch_expand(int op, const void* x, int M, int K, int g, int8_t* xq, float* amax, cudaStream_t s)
 {
     const long long warps = static_cast<long long>(M) * (K / g);
@@ -449,10 +485,19 @@ w4a16_status launch_expand(int op, const void* x, int M, int K, int g, int8_t* x
     const int v = g / 32;
     if (!(v == 1 || v == 2 || v == 4 || v == 8 || v == 12 || v == 16)) return W4A16_ERR_UNSUPPORTED;
     cudaError_t e;
-    switch (op_steps(op)) {
-        case 2: e = launch_expand_s<2>(blocks, xh, M, K, g, xq, amax, s); break;
-        case 4: e = launch_expand_s<4>(blocks, xh, M, K, g, xq, amax, s); break;
-        default: e = launch_expand_s<3>(blocks, xh, M, K, g, xq, amax, s); break;
+    if (g <= 256) {
+        // groups of up to 256 values: the 16-byte-per-thread form
+        switch (op_steps(op)) {
+            case 2: e = launch_expand8_s<2>(xh, M, K, g, xq, amax, s); break;
+            case 4: e = launch_expand8_s<4>(xh, M, K, g, xq, amax, s); break;
+            default: e = launch_expand8_s<3>(xh, M, K, g, xq, amax, s); break;
+        }
+    } else {
+        switch (op_steps(op)) {
+            case 2: e = launch_expand_s<2>(blocks, xh, M, K, g, xq, amax, s); break;
+            case 4: e = launch_expand_s<4>(blocks, xh, M, K, g, xq, amax, s); break;
+            default: e = launch_expand_s<3>(blocks, xh, M, K, g, xq, amax, s); break;
+        }
     }
     if (e != cudaSuccess) {
         (void)cudaGetLastError();

@@ -115,16 +115,6 @@ __device__ __forceinline__ uint32_t ldg_stream32(const void* p)
     return v;
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-// all but the N most recent groups of this thread's copies are complete
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
 // D += A . B on an m16n8k32 tile: A signed bytes, B unsigned bytes, int32
 // sums.  The fragments are whole register tuples (a[1] and a[3], rows 8-15,
 // stay zero), so no moves are needed around the instruction.

@@ -7,7 +7,7 @@
 //   repack_kernel   offline int4 re-layout (the "Marlin layout" idea,
 //                   pwwt.cn/news/2290475 section 6.2; QUICK's offline
 //                   interleave, briefgpt.xyz "QUICK" abstract).
-//   expand_kernel   MSD equations 1-8: A_max and the residual digits A1..A3
+//   expand8_kernel / expand_kernel   MSD equations 1-8: A_max and the residual digits A1..A3
 //                   (section 4.1, steps 1-8), written once to HBM.
 //   gemm_kernel     the tensor-core matmul, both variants, dense / split-K /
 //                   grouped-expert.  MSD: equations 9-11; DEQUANT: y = x.W'.
@@ -439,6 +439,89 @@ __global__ void __launch_bounds__(256) expand_kernel(const __half* __restrict__ 
             for (int p = 0; p < S; ++p) xq[p * plane + base + i] = d[p][i];
     }
     if (lane == 0) amax[static_cast<size_t>(gi) * M + m] = am;
+}
+
+// The same steps for g <= 256, shaped for memory-level parallelism.  A thread
+// takes 8 consecutive values (one 16-byte load) of the activations read as
+// one flat [M * K] array, so LPG = g / 8 threads share a group (A_max by a
+// shuffle over them; K % g == 0 keeps every group inside one row).  A warp
+// task is STEPS consecutive 256-value blocks whose loads are all issued
+// before any arithmetic; warps loop over tasks.  Each digit is rounded by
+// adding and subtracting 1.5 * 2^23: for |t| < 2^22 the sum falls where
+// binary32 values are the integers, so round-to-nearest-even there is rint(t)
+// and the subtraction is exact (every step here has |t| < 8).  The digit's
+// byte is then the low byte of the sum's bits (0x4B400000 + d).
+__device__ __forceinline__ uint32_t low_bytes4(float a, float b, float c, float d)
+{
+    const uint32_t lo = __byte_perm(__float_as_uint(a), __float_as_uint(b), 0x0040);
+    const uint32_t hi = __byte_perm(__float_as_uint(c), __float_as_uint(d), 0x0040);
+    return __byte_perm(lo, hi, 0x5410);
+}
+
+template <int LPG, int S, int STEPS>
+__global__ void __launch_bounds__(256) expand8_kernel(const __half* __restrict__ x, int M, int K, int g,
+                                                      int8_t* __restrict__ xq, float* __restrict__ amax)
+{
+    static_assert(LPG == 4 || LPG == 8 || LPG == 16 || LPG == 32, "g = 8 * LPG, 32 <= g <= 256");
+    // as expand_kernel: the consumer may launch now; wait for the producer of
+    // x and for the previous reader of xq
+    griddep_launch_dependents();
+    griddep_wait();
+    const int G = K / g;
+    const long long total8 = static_cast<long long>(M) * K / 8;    // 8-value vectors
+    const long long ntask = (total8 + 32 * STEPS - 1) / (32 * STEPS);
+    const int lane = threadIdx.x & 31;
+    const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+    const size_t plane = static_cast<size_t>(M) * K;
+    constexpr float kMagic = 12582912.0f;                          // 1.5 * 2^23
+    for (long long task = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) >> 5; task < ntask;
+         task += nwarps) {
+        uint4 raw[STEPS];
+#pragma unroll
+        for (int st = 0; st < STEPS; ++st) {
+            const long long v = (task * STEPS + st) * 32 + lane;
+            raw[st] = v < total8 ? __ldg(reinterpret_cast<const uint4*>(x + v * 8)) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int st = 0; st < STEPS; ++st) {
+            const long long v = (task * STEPS + st) * 32 + lane;
+            float f[8];
+            {
+                const uint32_t w[4] = {raw[st].x, raw[st].y, raw[st].z, raw[st].w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&w[h]));
+                    f[2 * h] = t.x;
+                    f[2 * h + 1] = t.y;
+                }
+            }
+            float am = 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(f[i]));
+#pragma unroll
+            for (int o = LPG / 2; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+            if (v >= total8) continue;       // whole groups lie past the end
+            float sv[S][8];                  // 1.5 * 2^23 + digit
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                float t = am == 0.f ? 0.f : __fdiv_rn(__fmul_rn(7.49f, f[i]), am);
+#pragma unroll
+                for (int p = 0; p < S; ++p) {
+                    sv[p][i] = __fadd_rn(t, kMagic);
+                    if (p + 1 < S) t = __fmul_rn(__fsub_rn(t, __fsub_rn(sv[p][i], kMagic)), 14.98f);
+                }
+            }
+#pragma unroll
+            for (int p = 0; p < S; ++p)
+                *reinterpret_cast<uint2*>(xq + p * plane + v * 8) =
+                    make_uint2(low_bytes4(sv[p][0], sv[p][1], sv[p][2], sv[p][3]),
+                               low_bytes4(sv[p][4], sv[p][5], sv[p][6], sv[p][7]));
+            if (lane % LPG == 0) {
+                const long long f0 = (v * 8) / g;                     // flat group index = m * G + gi
+                amax[static_cast<size_t>(f0 % G) * M + f0 / G] = am;
+            }
+        }
+    }
 }
 
 // ------------------------------------------------------------------ the tensor-core matmul
