@@ -366,10 +366,12 @@ w4a16_status launch_gemm(const CUtensorMap& map, const GemmParams& P, dim3 grid,
 //     thread for far longer than the tensor core needs (two issuers with
 //     more operand stages measured 40 % slower); two epilogue groups take
 //     alternate K groups; 16 activation stages of their own
-//   larger M:         MSD <64, 4, 4, 2, 2, 1>   DEQUANT <128, 4, 4, 2, 1, 2>
-//     two converter groups; MSD's per-group combine needs two epilogue
-//     groups; DEQUANT two issuers, each into its own accumulator
-//     (<256, 2, 4, 2, 2, 1> when there are enough tiles)
+//   larger M:         MSD <64, 4, 4, 1, 4, 1>   DEQUANT <128, 4, 4, 2, 1, 2>
+//     MSD: four epilogue groups of 16 tokens, each reading all of a group's
+//     sums before handing the buffer back (measured at prefill: 463 ->
+//     452 us against two groups of 32 tokens), one converter group (the
+//     warps that fit beside them); DEQUANT two issuers, each into its own
+//     accumulator (<256, 2, 4, 2, 2, 1> when there are enough tiles)
 //   bf16 dequant: <16, 4, 12, 2, 2, 4, scale in epilogue> and
 //     <128, 4, 4, 2, 2, 2, scale in epilogue>
 w4a16_status launch_for(int op, int TT, const CUtensorMap& map, const GemmParams& P, dim3 grid, cudaStream_t s)
@@ -379,18 +381,18 @@ w4a16_status launch_for(int op, int TT, const CUtensorMap& map, const GemmParams
         // with the window writes switched on
         if (P.dbg_yint != nullptr) {
             if (TT == 16) return launch_gemm<kMsd, 16, 8, 12, 2, 2, 4, false, true>(map, P, grid, s);
-            return launch_gemm<kMsd, 64, 4, 4, 2, 2, 1, false, true>(map, P, grid, s);
+            return launch_gemm<kMsd, 64, 4, 4, 1, 4, 1, false, true>(map, P, grid, s);
         }
         if (TT == 16) return launch_gemm<kMsd, 16, 8, 12, 2, 2, 4, false>(map, P, grid, s);
-        return launch_gemm<kMsd, 64, 4, 4, 2, 2, 1, false>(map, P, grid, s);
+        return launch_gemm<kMsd, 64, 4, 4, 1, 4, 1, false>(map, P, grid, s);
     }
     if (op == W4A16_OP_MSD_2STEP) {
         if (P.dbg_yint != nullptr) {
             if (TT == 16) return launch_gemm<kMsd2, 16, 8, 12, 2, 2, 4, false, true>(map, P, grid, s);
-            return launch_gemm<kMsd2, 64, 4, 4, 2, 2, 1, false, true>(map, P, grid, s);
+            return launch_gemm<kMsd2, 64, 4, 4, 1, 4, 1, false, true>(map, P, grid, s);
         }
         if (TT == 16) return launch_gemm<kMsd2, 16, 8, 12, 2, 2, 4, false>(map, P, grid, s);
-        return launch_gemm<kMsd2, 64, 4, 4, 2, 2, 1, false>(map, P, grid, s);
+        return launch_gemm<kMsd2, 64, 4, 4, 1, 4, 1, false>(map, P, grid, s);
     }
     if (op == W4A16_OP_MSD_4STEP) {
         // 4 x 16-row activation stages: 8 weight stages keep shared memory in bounds

@@ -164,6 +164,9 @@ struct GemmCfg {
     // split the tokens
     static constexpr bool kEpiRR = TT == 16 && NEPI > 1;
     static constexpr int kTokPerEpi = kEpiRR ? TT : TT / NEPI;
+    // MSD epilogue with at most 48 sums per thread and group: read them all,
+    // hand the buffer back, then combine
+    static constexpr bool kEpiBurst = kIsMsd && kTokPerEpi * kVals <= 48;
     static constexpr int kRedBytes = TT == 16 ? TT * kBN * 4 + 256 : 0;     // split-K partials (decode tile only)
     static constexpr int kRRBytes = kEpiRR ? (NEPI - 1) * TT * kBN * 4 : 0; // partial sums of groups 1..NEPI-1
     static constexpr int kNumBars = 2 * kBST + 2 * ST + 2 * WST + 2 * kNBuf + kMaxIssuers;
@@ -974,17 +977,15 @@ W4A16_ROLE_UNROLL
                 if (!ok) continue;
                 tc_fence_after();
                 const uint32_t b_addr = t_addr + ab * C::kAccStride + tb;
+                bool released = false;
                 if (C::kIsMsd) {
                     const float scc = sc * kC1;
-#pragma unroll
-                    for (int c = 0; c < TE / 8; ++c) {
-                        uint32_t yv[C::kVals][8];   // Y1..YS of 8 tokens
-#pragma unroll
-                        for (int p = 0; p < C::kVals; ++p) tmem_ld8(b_addr + p * TT + 8 * c, yv[p]);
+                    // equations 10-11 for 8 tokens of this column, and the
+                    // debug window's copy of their Y_i and A_max
+                    auto combine8 = [&](int c, const uint32_t (&yv)[C::kVals][8]) {
                         const float4 a0 = reinterpret_cast<const float4*>(am_slot + tb + 8 * c)[0];
                         const float4 a1 = reinterpret_cast<const float4*>(am_slot + tb + 8 * c)[1];
                         const float am[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-                        tmem_ld_wait();
 #pragma unroll
                         for (int qq = 0; qq < 8; qq += 2) {
                             float2 v = make_float2(__int2float_rn(static_cast<int>(yv[0][qq])),
@@ -1016,6 +1017,33 @@ W4A16_ROLE_UNROLL
                                 }
                             }
                         }
+                    };
+                    if constexpr (C::kEpiBurst) {
+                        // all of the group's sums into registers at once, then
+                        // the buffer goes back to the MMA before the combine:
+                        // the next group's MMAs run without this warp's
+                        // Tensor Memory reads beside them
+                        uint32_t yv[TE / 8][C::kVals][8];
+#pragma unroll
+                        for (int c = 0; c < TE / 8; ++c)
+#pragma unroll
+                            for (int p = 0; p < C::kVals; ++p) tmem_ld8(b_addr + p * TT + 8 * c, yv[c][p]);
+                        tmem_ld_wait();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(smem_addr(&accempty_bar[ab]));
+                        released = true;
+#pragma unroll
+                        for (int c = 0; c < TE / 8; ++c) combine8(c, yv[c]);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < TE / 8; ++c) {
+                            uint32_t yv[C::kVals][8];   // Y1..YS of 8 tokens
+#pragma unroll
+                            for (int p = 0; p < C::kVals; ++p) tmem_ld8(b_addr + p * TT + 8 * c, yv[p]);
+                            tmem_ld_wait();
+                            combine8(c, yv);
+                        }
                     }
                 } else {
 #pragma unroll
@@ -1027,9 +1055,11 @@ W4A16_ROLE_UNROLL
                         for (int k = 0; k < 16; ++k) acc[16 * c + k] = fmaf(__uint_as_float(v[k]), sc, acc[16 * c + k]);
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_addr(&accempty_bar[ab]));
+                if (!released) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_addr(&accempty_bar[ab]));
+                }
             }
             if (C::kEpiRR) {
                 // groups 1..NEPI-1 hand their partial sums to group 0, which
