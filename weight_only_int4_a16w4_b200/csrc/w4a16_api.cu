@@ -117,6 +117,39 @@ CUtensorMapDataType act_dtype(int op)
     return op == W4A16_OP_DEQUANT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
 }
 
+// The decode tile's activations, kBCopyGroup chunks per box (dense calls with
+// K % 128 == 0).  MSD: the digit planes [S][M][K] int8 seen as dims (128 k
+// of a chunk, row, plane, chunk); dequant: x [M][K] 16-bit as (64 k of a
+// half-chunk, row, half-chunk).  A box lands as kBCopyGroup consecutive
+// operand stages, each laid out as the two-dimensional boxes lay one out.
+bool make_map_grouped(CUtensorMap* map, const void* base, int op, int M, int K, int box_rows)
+{
+    auto fn = encode_fn();
+    if (!fn || K % kKC != 0) return false;
+    CUresult r;
+    if (is_msd_op(op)) {
+        const int S = op_steps(op);
+        cuuint64_t dims[4] = {static_cast<cuuint64_t>(kKC), static_cast<cuuint64_t>(M), static_cast<cuuint64_t>(S),
+                              static_cast<cuuint64_t>(K / kKC)};
+        cuuint64_t strides[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M) * K,
+                                 static_cast<cuuint64_t>(kKC)};
+        cuuint32_t box[4] = {static_cast<cuuint32_t>(kKC), static_cast<cuuint32_t>(box_rows),
+                             static_cast<cuuint32_t>(S), static_cast<cuuint32_t>(kBCopyGroup)};
+        cuuint32_t estr[4] = {1, 1, 1, 1};
+        r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    } else {
+        cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(M), static_cast<cuuint64_t>(K / 64)};
+        cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * 2, 128};
+        cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(2 * kBCopyGroup)};
+        cuuint32_t estr[3] = {1, 1, 1};
+        r = fn(map, act_dtype(op), 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    }
+    return r == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------- launch shapes
 
 struct Shape {
@@ -530,6 +563,7 @@ void base_params(GemmParams& P, int op, int M, int K, int N, int g, const Shape&
     P.status = static_cast<uint32_t*>(ws);
     P.timeout_ns = g_timeout_ns.load();
     P.write_y = 1;
+    P.bgroup = 1;
 }
 
 template <int VAR, int MR, bool DBG = false>
@@ -788,10 +822,12 @@ w4a16_status dense_matmul(int op, const void* x, const void* w_packed, const voi
         st = launch_expand(op, x, M, K, g, xq, amax, stream);
         if (st != W4A16_OK) return st;
         P.amax = amax;
-        if (!make_map(&map, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, op_steps(op) * M, kKC, s.TT))
+        if (s.TT == 16 && make_map_grouped(&map, xq, op, M, K, s.TT)) P.bgroup = kBCopyGroup;
+        else if (!make_map(&map, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, op_steps(op) * M, kKC, s.TT))
             return W4A16_ERR_CUDA;
     } else {
-        if (!make_map(&map, x, act_dtype(op), 2, K, M, 64, s.TT)) return W4A16_ERR_CUDA;
+        if (s.TT == 16 && make_map_grouped(&map, x, op, M, K, s.TT)) P.bgroup = kBCopyGroup;
+        else if (!make_map(&map, x, act_dtype(op), 2, K, M, 64, s.TT)) return W4A16_ERR_CUDA;
     }
     // four MMA issuers on the decode tile when a group is exactly one
     // 128-deep chunk: each issuer then owns one of the per-group

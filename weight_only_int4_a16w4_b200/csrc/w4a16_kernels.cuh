@@ -53,6 +53,12 @@ constexpr int kKC = 128;                 // K per pipeline stage
 constexpr int kWStage = kBN * kKC / 2;   // packed bytes per (tile, chunk): 8192
 constexpr int kMaxExperts = 64;
 constexpr int kMaxGroupMsd = 512;        // expand_kernel: at most 16 values per lane
+// Decode tile: chunks per bulk copy of weights, and per tensor copy of
+// activations when the map allows it.  Fewer, larger copies: the producers
+// otherwise issue one chunk's copies per loop pass, and a pass costs far more
+// than its few instructions (about 0.4 us per chunk measured on B200).
+constexpr int kWCopyGroup = 4;          // weight chunks per bulk copy
+constexpr int kBCopyGroup = 4;          // activation chunks per tensor copy
 
 // kDeqBf16: the dequant variant with bf16 x, scale and y (the INT4 + BF16
 // pairing of the Humming article, aihirek.info).  Its buffers travel in the
@@ -98,6 +104,9 @@ struct GemmParams {
     uint32_t* status;
     unsigned long long timeout_ns;
     int write_y;
+    // decode tile: chunks per activation copy (1, or kBCopyGroup when the
+    // tensor map spans kBCopyGroup chunks per box: dense calls, K % 128 == 0)
+    int bgroup;
     int32_t* dbg_yint;                      // MSD debug window (or nullptr)
     float* dbg_amax;
     int dbg_m0, dbg_m1, dbg_n0, dbg_n1;
@@ -141,6 +150,10 @@ struct GemmCfg {
     // L2 latency off the MMA's path; elsewhere one per operand stage
     static constexpr int kBST = TT == 16 ? 16 : ST;
     static constexpr int kWSlot = kWStage + kSBytes;                       // weight stage
+    // weight chunks per bulk copy: a tile's packed blocks of consecutive
+    // chunks are contiguous, so with no scale rows in the slots one copy
+    // fills several (decode tile)
+    static constexpr int kWG = (TT == 16 && kSBytes == 0 && WST % kWCopyGroup == 0) ? kWCopyGroup : 1;
     static constexpr int kMaxIssuers = NISS;
     // accumulator buffers: per group (two, or one per issuer); a single
     // accumulator over all of K otherwise, one per issuer (added up, in
@@ -179,6 +192,7 @@ struct GemmCfg {
     static_assert(kSmem <= 227 * 1024, "shared memory overflow");
     static_assert(ST % NCONV == 0 && ST % NISS == 0 && WST % NCONV == 0 && kBST % NISS == 0,
                   "stages must split evenly over the groups");
+    static_assert(TT != 16 || kBST % kBCopyGroup == 0, "grouped activation copies never wrap the ring");
     static_assert(NISS == 1 || NISS == 2 || NISS == 4, "1, 2 or 4 MMA issuers");
     static_assert(!SEPI || !kIsMsd, "SEPI is a DEQUANT option");
     // bf16 keeps 8 significant bits: a product scale * w does not fit, so the
@@ -661,7 +675,46 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
             // commit frees both
             uint64_t* freeb = weights ? wempty_bar : (C::kBST == ST ? sfree_bar : bfree_bar);
             int issued = 0;
-            for (int i = 0; i < nchunks; ++i) {
+            // groups of gsz chunks: one copy into gsz consecutive slots (the
+            // ring is a multiple of gsz: a group never wraps), completing on
+            // the group's first slot's barrier; a short last group still
+            // lands a whole box (past the end: zero fill or chunks nobody
+            // reads), so every slot of it is waited free
+            const int gsz = weights ? C::kWG : (TT == 16 ? P.bgroup : 1);
+            if (gsz > 1) {
+                int groups = 0;
+                for (int i0 = 0; i0 < nchunks; i0 += gsz) {
+                    const int nc = min(gsz, nchunks - i0);
+                    const int s0 = i0 % ring;
+                    const uint32_t ph = (i0 / ring) & 1;
+                    bool free_ok = true;
+                    for (int c = 0; c < gsz && free_ok; ++c)
+                        free_ok = mbar_wait(smem_addr(&freeb[s0 + c]), ph ^ 1, tmo, P.status, abort_flag);
+                    if (!free_ok) break;
+                    if (lane == 0) {
+                        const uint32_t fb = smem_addr(&fullb[s0]);
+                        const int kc = kc0 + i0;
+                        if (weights) {
+                            mbar_arrive_expect_tx(fb, static_cast<uint32_t>(nc) * kWStage);
+                            bulk_g2s(smem_addr(wsm + s0 * C::kWSlot), wsrc + static_cast<size_t>(i0) * kWStage,
+                                     static_cast<uint32_t>(nc) * kWStage, fb);
+                        } else {
+                            mbar_arrive_expect_tx(fb, static_cast<uint32_t>(gsz) * C::kBBytes);
+                            if (C::kIsMsd) tma_load_4d(smem_addr(smem + s0 * C::kStage), &tmap, 0, tc.t0, 0, kc, fb);
+                            else tma_load_3d(smem_addr(smem + s0 * C::kStage), &tmap, 0, tc.t0, 2 * kc, fb);
+                        }
+                    }
+                    __syncwarp();
+                    ++groups;
+                }
+                // Drain: the last group issued on each first slot has landed.
+                const int gpr = ring / gsz;        // groups per ring cycle
+                for (int k0 = 0; k0 < gpr && k0 < groups; ++k0) {
+                    const int kl = k0 + ((groups - 1 - k0) / gpr) * gpr;
+                    mbar_wait(smem_addr(&fullb[k0 * gsz]), ((kl * gsz) / ring) & 1, tmo, P.status, nullptr);
+                }
+            }
+            for (int i = 0; i < nchunks && gsz == 1; ++i) {
                 const int s = i % ring;
                 const uint32_t ph = (i / ring) & 1;
                 if (!mbar_wait(smem_addr(&freeb[s]), ph ^ 1, tmo, P.status, abort_flag)) break;
@@ -736,7 +789,8 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
                 const int bs = i % C::kBST;
                 const uint32_t bph = (i / C::kBST) & 1;
                 if (!mbar_wait(smem_addr(&afull_bar[s]), ph, tmo, P.status, abort_flag)) break;
-                if (!mbar_wait(smem_addr(&bfull_bar[bs]), bph, tmo, P.status, abort_flag)) break;
+                // (grouped activation copies complete on the group's first slot)
+                if (!mbar_wait(smem_addr(&bfull_bar[bs - bs % P.bgroup]), bph, tmo, P.status, abort_flag)) break;
                 tc_fence_after();
                 const uint64_t bdesc = smem_desc_sw128(smem_addr(smem + bs * C::kStage));
                 const uint32_t a_base = tmem_a0 + s * C::kACols;
@@ -818,7 +872,8 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
             const uint32_t ph = (i / ST) & 1;
             const int w = i % WST;
             const uint32_t wph = (i / WST) & 1;
-            if (!mbar_wait(smem_addr(&wfull_bar[w]), wph, tmo, P.status, abort_flag)) break;
+            // the slot's copy completes on its group's first slot's barrier
+            if (!mbar_wait(smem_addr(&wfull_bar[w - w % C::kWG]), wph, tmo, P.status, abort_flag)) break;
             const uint8_t* wst = wsm + w * C::kWSlot;
             uint4 q[4];
 #pragma unroll
