@@ -789,8 +789,10 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
                 const int bs = i % C::kBST;
                 const uint32_t bph = (i / C::kBST) & 1;
                 if (!mbar_wait(smem_addr(&afull_bar[s]), ph, tmo, P.status, abort_flag)) break;
-                // (grouped activation copies complete on the group's first slot)
-                if (!mbar_wait(smem_addr(&bfull_bar[bs - bs % P.bgroup]), bph, tmo, P.status, abort_flag)) break;
+                // (grouped activation copies, decode tile only, complete on
+                // the group's first slot)
+                const int bfs = TT == 16 ? bs - bs % P.bgroup : bs;
+                if (!mbar_wait(smem_addr(&bfull_bar[bfs]), bph, tmo, P.status, abort_flag)) break;
                 tc_fence_after();
                 const uint64_t bdesc = smem_desc_sw128(smem_addr(smem + bs * C::kStage));
                 const uint32_t a_base = tmem_a0 + s * C::kACols;
@@ -814,6 +816,21 @@ __global__ void __launch_bounds__(GemmCfg<VAR, TT, ST, WST, NCONV, NEPI, NISS, S
                         else mma_f16_ts(d, a_base + 8 * j, bd, idesc, j == 0 ? 0u : 1u);
                     }
                     tc_commit(smem_addr(&accfull_bar[ab]));
+                    tc_commit(smem_addr(&sfree_bar[s]));
+                    if (C::kBST != ST) tc_commit(smem_addr(&bfree_bar[bs]));
+                    first_chunk = false;
+                    continue;
+                }
+                if (!C::kGroupAcc && nsteps == kSteps) {
+                    // a full chunk into the issuer's one accumulator: every
+                    // step's operands and flags known at compile time (the
+                    // issuing lane's loop is on the tensor pipe's critical path)
+                    const uint32_t d = tmem + q * C::kAccStride;
+#pragma unroll
+                    for (int j = 0; j < kSteps; ++j) {
+                        const uint64_t bd = C::kIsMsd ? bdesc + 2 * j : bdesc + ((j >> 2) * (TT * 128) >> 4) + 2 * (j & 3);
+                        mma_f16_ts(d, a_base + 8 * j, bd, idesc, (j == 0 && first_chunk) ? 0u : 1u);
+                    }
                     tc_commit(smem_addr(&sfree_bar[s]));
                     if (C::kBST != ST) tc_commit(smem_addr(&bfree_bar[bs]));
                     first_chunk = false;
