@@ -263,15 +263,14 @@ int gemv_mma_smem_nw_op(int op, int NW, int M, int K, int g)
 }
 
 // Warps per CTA of the warp-MMA GEMV.  Measured on B200 (us per call, 16 vs
-// 32 warps): dequant at M <= 2 gains from 32 warps of one quad-round each
-// (K 4096, N 14336: 17.3 -> 16.3; K = N = 8192: 18.2 -> 16.8; K = N = 4096:
-// 5.92 -> 5.84); for MSD 16 warps are faster (K 4096, N 14336: 14.7 vs 15.6;
-// K = N = 4096: 6.35 vs 6.8); 8 warps lose everywhere.
+// 32 warps): dequant at M <= 2 with N >= 8192 gains from 32 warps of one
+// quad-round each (K 4096, N 14336: 17.3 -> 16.3; K = N = 8192: 18.2 ->
+// 16.8); at N = 4096 and for MSD, 16 warps are as fast or faster (MSD
+// K 4096, N 14336: 14.7 vs 15.6); 8 warps lose everywhere.
 int gemv_mma_warps(int op, int M, int K, int N, int g)
 {
-    (void)N;
     int nw = 16;
-    if (!is_msd_op(op) && M <= 2) nw = 32;
+    if (!is_msd_op(op) && M <= 2 && N >= 8192) nw = 32;
     if (nw == 32 && gemv_mma_smem_nw_op(op, 32, M, K, g) > kMaxSmemOptin) nw = 16;
     return nw;
 }
