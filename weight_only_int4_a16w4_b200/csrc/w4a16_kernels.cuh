@@ -20,19 +20,23 @@
 // the B200 analogue of stacking A1..A3 into a 3M-row A_int (section 4.1
 // step 8; section 8.1 "singleCoreM = 3*M"), so one MMA produces Y1, Y2, Y3.
 //
-// Warp roles (320 threads):
-//   warp 0      producer: bulk-copies the packed weight chunk (and the fp16
-//               scale rows for DEQUANT) and TMA-loads the activation tile of
-//               each 128-deep K chunk into a ring of shared-memory stages.
-//   warp 1      Tensor Memory allocation; one thread issues the tcgen05 MMAs.
-//   warps 2-5   converters: shared-memory int4 -> MMA operand A in Tensor
-//               Memory (int8 for MSD, fp16 * scale for DEQUANT), one thread
-//               per weight row, written with tcgen05.st.
-//   warps 6-9   epilogue: tcgen05.ld of the accumulators; MSD combines
-//               Y1..Y3 with A_max and the scale after every group
-//               (equations 10-11) while the MMAs of the next group run
-//               (the PRELOAD_MSD overlap of section 6.2, done with
-//               double-buffered accumulators); fp16 store or split-K partial.
+// Warp roles (the counts are template parameters; GemmCfg below):
+//   warp 0      weight producer: bulk copies of the packed weight chunks
+//               (and the fp16 scale rows when the converter applies them)
+//               into a ring of shared-memory slots; four chunks per copy on
+//               the decode tile.
+//   warp 1      activation producer (TMA tiles of x, or of the digit planes,
+//               into the operand stages) and Tensor Memory allocation.
+//   warps 2..   MMA issuers: one lane each issues the tcgen05 MMAs of its
+//               chunks and commits them to the stage / accumulator barriers.
+//   converters  groups of 4 warps: shared-memory int4 -> MMA operand A in
+//               Tensor Memory (int8 for MSD, fp16 or bf16 for DEQUANT), one
+//               thread per weight row, written with tcgen05.st.
+//   epilogue    groups of 4 warps: tcgen05.ld of the accumulators; MSD
+//               combines Y1..Y3 with A_max and the scale after every group
+//               (equations 10-11) while the MMAs of the next group run (the
+//               PRELOAD_MSD overlap of section 6.2, done with multi-buffered
+//               accumulators); fp16 / bf16 store or split-K partial.
 #pragma once
 
 #ifndef W4A16_ROLE_UNROLL
